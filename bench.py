@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA prefill chunk (indexer -> exact top-k -> sparse MLA) on B200.
+
+One step = one dsa_prefill_chunk call over one synthetic chunk resident in HBM
+(default: the 128K-context workload, N = 131,072 cached keys, L = 1,024
+queries).  Prints one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Timing: W untimed warm-up steps; then K steps, each preceded by a 512 MiB
+device write that flushes the 126 MB L2, each bracketed by CUDA events on the
+launching stream (the flush is outside the events); a barrier and a device
+synchronise on both sides of the timed region; max over ranks.  With N > 1
+every rank runs an independent replica (the path has no cross-GPU exchange):
+value = all ranks' query tokens / max rank time (weak scaling).
+
+--impl reference times the CPU oracle (the plain fp64 C implementation the
+tests compare against) on the host cores, on a bounded sample of the same
+workload's queries.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import dsa_inputs  # noqa: E402
+
+METRIC = "DSA prefill query tokens/s at 128K ctx (indexer+top-k+sparse MLA); % roofline"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 512 << 20
+EVENTS_PER_BLOCK = 7
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def indexer_kernel_traffic(cfg) -> int | None:
+    """DRAM bytes per launch of the main indexer kernel from the committed ncu summary, if it still applies."""
+    path = os.path.join(ROOT, "profiles", "indexer_main_traffic.txt")
+    src = os.path.join(ROOT, "deepseek_sparse_attention_relu_b200", "csrc", "indexer.cu")
+    if not os.path.exists(path):
+        return None
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("indexer_cu_sha256_16") != sha or vals.get("workload") != cfg.name:
+        return None
+    try:
+        return int(float(vals["dram_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples (every 200 ms) while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_rate(cfg, inp, rows: list[int], threads: int) -> tuple[float, float]:
+    """Query tokens/s of the unmodified oracle over `rows` on `threads` host threads; returns (rate, seconds)."""
+    import oracle
+    pb = oracle.Problem(dsa_inputs.raw_bits(inp["q_idx"]), dsa_inputs.raw_bits(inp["k_idx"]), inp["w"],
+                        cfg.idx_code, cfg.L, cfg.N, cfg.H_I, cfg.D_I, cfg.q_pos0, cfg.topk,
+                        q=dsa_inputs.raw_bits(inp["q"]), kv=dsa_inputs.raw_bits(inp["kv"]), H=cfg.H, scale=cfg.scale)
+    t0 = time.perf_counter()
+    oracle.map_rows(lambda t: oracle.prefill_row(pb, t), rows, threads=threads)
+    dt = time.perf_counter() - t0
+    return len(rows) / dt, dt
+
+
+def sample_rows(cfg, n: int, salt: int = 0) -> list[int]:
+    g = torch.Generator().manual_seed(1234 + salt)
+    return sorted(torch.randperm(cfg.L, generator=g)[:min(n, cfg.L)].tolist())
+
+
+def flops_and_bytes(cfg) -> dict:
+    pairs = cfg.visible_pairs()
+    idx_flop = pairs * 2 * cfg.H_I * cfg.D_I
+    mla_flop = cfg.L * cfg.H * cfg.topk * (576 + 512) * 2
+    esz = 1 if cfg.idx_dtype == "e4m3" else 2
+    alg_bytes = (cfg.N * cfg.D_I * esz + cfg.L * cfg.H_I * cfg.D_I * esz + cfg.L * cfg.H_I * 4
+                 + min(cfg.N, cfg.L * cfg.topk) * 1152 + cfg.L * cfg.H * 576 * 2 + cfg.L * cfg.H * 512 * 2
+                 + cfg.L * cfg.topk * 4)
+    return {"pairs": pairs, "indexer_flop": idx_flop, "mla_flop": mla_flop, "alg_bytes": alg_bytes}
+
+
+def run_reference(args, rank: int, world: int) -> None:
+    if rank != 0:
+        return
+    cfg = dsa_inputs.BY_NAME[args.workload]
+    inp = dsa_inputs.generate(cfg)
+    threads = os.cpu_count() or 1
+    rows_per_step = max(1, min(cfg.L, threads))
+    for w in range(args.warmup):
+        cpu_oracle_rate(cfg, inp, sample_rows(cfg, max(1, rows_per_step // 4), salt=100 + w), threads)
+    total_rows, total_s = 0, 0.0
+    for k in range(args.steps):
+        rows = sample_rows(cfg, rows_per_step, salt=k)
+        _, dt = cpu_oracle_rate(cfg, inp, rows, threads)
+        total_rows += len(rows)
+        total_s += dt
+    value = total_rows / total_s
+    sample = (f"{args.steps} steps x {rows_per_step} seeded-random query rows of the workload "
+              f"(full indexer row + exact top-k + attention per row)")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "N": cfg.N, "L": cfg.L, "topk": cfg.topk, "H": cfg.H, "H_I": cfg.H_I,
+                   "D_I": cfg.D_I, "indexer_dtype": cfg.idx_dtype, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }), flush=True)
+
+
+def run_ours(args, rank: int, world: int, local_rank: int) -> None:
+    import deepseek_sparse_attention_relu_b200 as dsa
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    cfg = dsa_inputs.BY_NAME[args.workload]
+    t_gen = time.perf_counter()
+    inp = dsa_inputs.generate(cfg)
+    log(f"[bench] rank {rank}: generated {cfg.name} in {time.perf_counter() - t_gen:.1f}s")
+    g = {k: v.to(dev) for k, v in inp.items()}
+    out = torch.empty(cfg.L, cfg.H, 512, dtype=torch.bfloat16, device=dev)
+    dt = dsa.DSA_BF16 if cfg.idx_dtype == "bf16" else dsa.DSA_FP8_E4M3
+    ws = dsa.alloc_workspace(dsa.dsa_prefill_chunk_workspace(cfg.L, cfg.N, cfg.H_I, cfg.D_I, cfg.H, cfg.topk, 0, dt,
+                                                             False), dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    nblocks = (cfg.L + 1023) // 1024
+    stream = torch.cuda.current_stream()
+
+    def new_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record(stream)  # materialise the handle
+        return evs
+
+    def step(events):
+        dsa.dsa_prefill_chunk_profiled(g["q_idx"], g["k_idx"], g["w"], g["q"], g["kv"], cfg.q_pos0, cfg.topk,
+                                       cfg.scale, out, events, workspace=ws)
+
+    warm_ev = new_events(EVENTS_PER_BLOCK * nblocks)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(warm_ev)
+    torch.cuda.synchronize()
+    status = dsa.dsa_workspace_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status word {status:#x} after warm-up")
+
+    starts = new_events(args.steps)
+    ends = new_events(args.steps)
+    stage_ev = [new_events(EVENTS_PER_BLOCK * nblocks) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.zero_()
+        starts[k].record(stream)
+        step(stage_ev[k])
+        ends[k].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    status = dsa.dsa_workspace_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status word {status:#x} after the timed steps")
+
+    step_ms = [starts[k].elapsed_time(ends[k]) for k in range(args.steps)]
+    total_ms = sum(step_ms)
+    # per-stage times (ms per step, summed over query blocks)
+    stage_names = ["pilot", "threshold", "indexer_main", "select", "fallback", "mla"]
+    stages = {n: 0.0 for n in stage_names}
+    main_launch_ms = []
+    for k in range(args.steps):
+        for b in range(nblocks):
+            ev = stage_ev[k][EVENTS_PER_BLOCK * b: EVENTS_PER_BLOCK * (b + 1)]
+            for i, n in enumerate(stage_names):
+                stages[n] += ev[i].elapsed_time(ev[i + 1]) / args.steps
+            main_launch_ms.append(ev[2].elapsed_time(ev[3]))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * cfg.L * args.steps / (total_ms / 1000.0)
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
+    host = {k: v.pin_memory() for k, v in inp.items()}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        for k2, v in host.items():
+            g[k2].copy_(v, non_blocking=True)
+        dsa.dsa_prefill_chunk(g["q_idx"], g["k_idx"], g["w"], g["q"], g["kv"], cfg.q_pos0, cfg.topk, cfg.scale,
+                              out, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * cfg.L * e2e_steps / (e2e_ms / 1000.0)
+
+    # ---- roofline of the dominant kernel (main indexer pass: tensor-core contraction)
+    fb = flops_and_bytes(cfg)
+    peaks = measured_peaks()
+    main_ms = statistics.mean(main_launch_ms)
+    launches_per_step = nblocks
+    idx_flop_per_launch = fb["indexer_flop"] / launches_per_step
+    achieved = idx_flop_per_launch / (main_ms / 1000.0) / 1e12
+    peak = peaks["bf16_tflops"] * (2.0 if cfg.idx_dtype == "e4m3" else 1.0)
+    traffic = indexer_kernel_traffic(cfg)
+    # whole-path roofline: max(tensor time at peak, algorithmic bytes at HBM bandwidth)
+    t_tensor = (fb["indexer_flop"] / (peak * 1e12)) + fb["mla_flop"] / (peaks["bf16_tflops"] * 1e12)
+    t_bytes = fb["alg_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    path_roof_s = max(t_tensor, t_bytes)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        n_rows = max(4, min(cfg.L, 6 * threads))
+        rows = sample_rows(cfg, n_rows)
+        rate, secs = cpu_oracle_rate(cfg, inp, rows, threads)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{len(rows)} seeded-random query rows of {cfg.name} (full indexer row, exact top-k, "
+                         f"attention), {secs:.1f} s wall on {threads} threads"}
+
+    pilot_launches = 1 if cfg.q_pos0 + min(cfg.L, 1024) > 8192 else 0
+    gpu_launches = args.steps * nblocks * (5 + pilot_launches)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.idx_dtype if cfg.idx_dtype == "bf16" else "fp8-e4m3 indexer / bf16 MLA",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "N": cfg.N, "L": cfg.L, "topk": cfg.topk, "H": cfg.H, "H_I": cfg.H_I,
+                   "D_I": cfg.D_I, "indexer_dtype": cfg.idx_dtype, "query_block": 1024,
+                   "l2": "flushed before every timed step (512 MiB device write, outside the step events)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "indexer_kernel (main pass)",
+                     "peak_source": f"{peaks['source']} bf16 burst" + (" x2 nominal fp8 ratio" if cfg.idx_dtype == "e4m3" else ""),
+                     "path_frac": path_roof_s / (ms_per_step / 1000.0)},
+        "stages_ms": {k: round(v, 4) for k, v in stages.items()},
+        "clocks": clocks,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": gpu_launches,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=dsa_inputs.CTX128K.name, choices=sorted(dsa_inputs.BY_NAME))
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        log(f"[bench] note: WORLD_SIZE={world} but --gpus={args.gpus}; using WORLD_SIZE")
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,451 @@
+// api.cu -- the C ABI of libdsa.so (declared in include/dsa.h): argument
+// checks, workspace carving, TMA descriptor encoding and the per-query-block
+// launch sequence of the DSA prefill path.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/dsa.h"
+#include "dsa_internal.h"
+
+namespace {
+
+using namespace dsa;
+
+constexpr int kDefaultQueryBlock = 1024;  // mlx-lm PR #1997: query blocks of 1,024
+constexpr int kSamples = 4096;            // strided key sample per query block
+constexpr int kFallbackSlots = 16;        // CTAs (and score rows) of the exact fallback
+constexpr int kMinCap = 8192;             // default candidate capacity per query
+constexpr int kMaxTopk = 4096;
+constexpr size_t kHeaderBytes = 256;      // status word, fallback counters
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  // The driver entry point is looked up once; it carries no per-call state.
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D tiled map: `rows` rows of `inner` elements, `pitch` bytes apart; box of
+// box_inner x box_rows elements, 128-byte swizzle, zero fill out of bounds.
+bool make_map_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t inner, uint64_t rows,
+                 uint64_t pitch, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  std::memset(m, 0, sizeof(*m));
+  return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+int default_cap(int topk) { return std::max(kMinCap, 4 * topk); }
+
+// Fixed part of the indexer workspace (everything but the candidate lists).
+size_t idx_fixed_bytes(int QB, int N) {
+  return kHeaderBytes + 3 * align256(static_cast<size_t>(QB) * 4) +
+         align256(static_cast<size_t>(QB) * kSamples * 4) + align256(static_cast<size_t>(kFallbackSlots) * N * 4);
+}
+
+struct IdxWorkspace {
+  unsigned *status;
+  int *fb_counters;
+  unsigned *tau;
+  int *cand_count;
+  int *fb_list;
+  float *dense;
+  float *fb_scratch;
+  unsigned long long *cand;
+  int cap;
+};
+
+bool carve_idx_ws(void *ws, size_t bytes, int QB, int N, IdxWorkspace *o) {
+  const size_t fixed = idx_fixed_bytes(QB, N);
+  if (ws == nullptr || bytes < fixed + static_cast<size_t>(QB) * 8) return false;
+  uint8_t *p = static_cast<uint8_t *>(ws);
+  o->status = reinterpret_cast<unsigned *>(p);
+  o->fb_counters = reinterpret_cast<int *>(p + 16);
+  p += kHeaderBytes;
+  o->tau = reinterpret_cast<unsigned *>(p);
+  p += align256(static_cast<size_t>(QB) * 4);
+  o->cand_count = reinterpret_cast<int *>(p);
+  p += align256(static_cast<size_t>(QB) * 4);
+  o->fb_list = reinterpret_cast<int *>(p);
+  p += align256(static_cast<size_t>(QB) * 4);
+  o->dense = reinterpret_cast<float *>(p);
+  p += align256(static_cast<size_t>(QB) * kSamples * 4);
+  o->fb_scratch = reinterpret_cast<float *>(p);
+  p += align256(static_cast<size_t>(kFallbackSlots) * N * 4);
+  o->cand = reinterpret_cast<unsigned long long *>(p);
+  const size_t room = (bytes - fixed) / (static_cast<size_t>(QB) * 8);
+  o->cap = static_cast<int>(std::min<size_t>(room, 1u << 30));
+  return o->cap >= 1;
+}
+
+struct IndexerProblem {
+  const void *q_idx, *k_idx;
+  const float *w;
+  bool fp8;
+  int L, N, H_I, D_I, q_pos0, topk;
+  int32_t *topk_idx;
+  float *topk_score;
+};
+
+dsa_status_t check_indexer_args(const IndexerProblem &p) {
+  if (p.q_idx == nullptr || p.k_idx == nullptr || p.w == nullptr || p.topk_idx == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(p.q_idx) || !aligned16(p.k_idx) || !aligned16(p.w) || !aligned16(p.topk_idx))
+    return DSA_ERR_INVALID_ARG;
+  if (p.topk_score != nullptr && !aligned16(p.topk_score)) return DSA_ERR_INVALID_ARG;
+  if (p.L <= 0 || p.N <= 0 || p.H_I <= 0 || p.D_I <= 0 || p.topk <= 0 || p.q_pos0 < 0) return DSA_ERR_INVALID_ARG;
+  if (static_cast<long long>(p.q_pos0) + p.L > p.N) return DSA_ERR_INVALID_ARG;
+  if (p.topk > kMaxTopk) return DSA_ERR_UNSUPPORTED;
+  if (!indexer_supported(p.D_I, p.H_I, p.fp8)) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+// Stages 1+2 for queries [t0, t0 + Lb) of the chunk.
+// Record ev[i] on the stream when profiling events were supplied.
+bool mark(cudaEvent_t *ev, int i, cudaStream_t stream) {
+  return ev == nullptr || ev[i] == nullptr || cudaEventRecord(ev[i], stream) == cudaSuccess;
+}
+
+// ev (optional): 6 events recorded before the pilot, after the pilot, after the
+// threshold, after the main indexer pass, after the selection, after the fallback.
+dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, const CUtensorMap &tk,
+                               const IdxWorkspace &ws, int t0, int Lb, cudaStream_t stream,
+                               cudaEvent_t *ev = nullptr) {
+  const int QG = indexer_queries_per_group(p.H_I);
+  const int G = (Lb + QG - 1) / QG;
+  const int q_pos0 = p.q_pos0 + t0;
+  const int sms = std::max(1, sm_count());
+  const long long esz = p.fp8 ? 1 : 2;
+  const long long row_bytes = static_cast<long long>(p.D_I) * esz;
+
+  IndexerArgs ia{};
+  ia.w = p.w + static_cast<long long>(t0) * p.H_I;
+  ia.tau = ws.tau;
+  ia.dense = ws.dense;
+  ia.cand = ws.cand;
+  ia.cand_count = ws.cand_count;
+  ia.status = ws.status;
+  ia.cap = ws.cap;
+  ia.Lb = Lb;
+  ia.q_pos0 = q_pos0;
+  ia.q_row0 = t0 * p.H_I;
+
+  const bool pilot = static_cast<long long>(q_pos0) + Lb > ws.cap;
+  int n_samples = 0;
+  if (!mark(ev, 0, stream)) return DSA_ERR_CUDA;
+  if (pilot) {
+    n_samples = std::min(kSamples, q_pos0 + 1);
+    const long long stride = (static_cast<long long>(q_pos0) + 1) / n_samples;
+    CUtensorMap ts;
+    const CUtensorMapDataType dt = p.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_map_2d(&ts, p.k_idx, dt, p.D_I, n_samples, stride * row_bytes, 128 / esz, 128)) return DSA_ERR_CUDA;
+    IndexerArgs pa = ia;
+    pa.pilot = 1;
+    pa.dense_ld = n_samples;
+    pa.n_keys = n_samples;
+    pa.total_tiles = G * ((n_samples + 127) / 128);
+    if (launch_indexer(tq, ts, pa, p.D_I, p.H_I, p.fp8, true, std::min(sms, pa.total_tiles), stream) !=
+        cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
+
+  SelectArgs sa{};
+  sa.q_idx = p.q_idx;
+  sa.k_idx = p.k_idx;
+  sa.w = p.w;
+  sa.dense = pilot ? ws.dense : nullptr;
+  sa.tau = ws.tau;
+  sa.cand = ws.cand;
+  sa.cand_count = ws.cand_count;
+  sa.fb_list = ws.fb_list;
+  sa.fb_counters = ws.fb_counters;
+  sa.fb_scratch = ws.fb_scratch;
+  sa.status = ws.status;
+  sa.topk_idx = p.topk_idx;
+  sa.topk_score = p.topk_score;
+  sa.dense_ld = n_samples;
+  sa.n_samples = n_samples;
+  sa.cap = ws.cap;
+  sa.fb_slots = kFallbackSlots;
+  sa.t0 = t0;
+  sa.Lb = Lb;
+  sa.q_pos0 = q_pos0;
+  sa.N = p.N;
+  sa.H_I = p.H_I;
+  sa.D_I = p.D_I;
+  sa.topk = p.topk;
+  sa.fp8 = p.fp8 ? 1 : 0;
+  if (!mark(ev, 1, stream)) return DSA_ERR_CUDA;
+  if (launch_threshold(sa, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!mark(ev, 2, stream)) return DSA_ERR_CUDA;
+
+  IndexerArgs ea = ia;
+  ea.pilot = 0;
+  ea.n_keys = p.N;
+  long long total = 0;
+  for (int g = 0; g < G; ++g) {
+    const int last = std::min(Lb, (g + 1) * QG);
+    const long long keys = std::min<long long>(p.N, static_cast<long long>(q_pos0) + last);
+    total += (keys + 127) / 128;
+  }
+  if (total > (1ll << 30)) return DSA_ERR_UNSUPPORTED;
+  ea.total_tiles = static_cast<int>(total);
+  if (launch_indexer(tq, tk, ea, p.D_I, p.H_I, p.fp8, false, static_cast<int>(std::min<long long>(sms, total)),
+                     stream) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (!mark(ev, 3, stream)) return DSA_ERR_CUDA;
+  if (launch_select(sa, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!mark(ev, 4, stream)) return DSA_ERR_CUDA;
+  if (launch_fallback(sa, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!mark(ev, 5, stream)) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+bool make_indexer_maps(const IndexerProblem &p, CUtensorMap *tq, CUtensorMap *tk) {
+  const CUtensorMapDataType dt = p.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint32_t esz = p.fp8 ? 1 : 2;
+  const uint64_t row_bytes = static_cast<uint64_t>(p.D_I) * esz;
+  return make_map_2d(tq, p.q_idx, dt, p.D_I, static_cast<uint64_t>(p.L) * p.H_I, row_bytes, 128 / esz, 256) &&
+         make_map_2d(tk, p.k_idx, dt, p.D_I, p.N, row_bytes, 128 / esz, 128);
+}
+
+struct MlaProblem {
+  const void *q, *kv;
+  const int32_t *topk_idx;
+  int L, N, H, topk;
+  float scale;
+  void *out;
+  float *lse;
+};
+
+dsa_status_t check_mla_args(const MlaProblem &p) {
+  if (p.q == nullptr || p.kv == nullptr || p.topk_idx == nullptr || p.out == nullptr) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(p.q) || !aligned16(p.kv) || !aligned16(p.topk_idx) || !aligned16(p.out))
+    return DSA_ERR_INVALID_ARG;
+  if (p.lse != nullptr && !aligned16(p.lse)) return DSA_ERR_INVALID_ARG;
+  if (p.L <= 0 || p.N <= 0 || p.H <= 0 || p.topk <= 0) return DSA_ERR_INVALID_ARG;
+  if (!std::isfinite(p.scale)) return DSA_ERR_INVALID_ARG;
+  if (static_cast<long long>(p.L) * p.H >= (1ll << 31)) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+bool make_mla_maps(const MlaProblem &p, CUtensorMap *tq, CUtensorMap *tkv) {
+  return make_map_2d(tq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 576, static_cast<uint64_t>(p.L) * p.H, 576 * 2, 64,
+                     64) &&
+         make_map_2d(tkv, p.kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 576, p.N, 576 * 2, 64, 1);
+}
+
+dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, const CUtensorMap &tkv, unsigned *status,
+                           int t0, int Lq, cudaStream_t stream) {
+  MlaArgs a{};
+  a.topk_idx = p.topk_idx;
+  a.out = static_cast<uint16_t *>(p.out);
+  a.lse = p.lse;
+  a.status = status;
+  a.L = p.L;
+  a.N = p.N;
+  a.H = p.H;
+  a.topk = p.topk;
+  a.t0 = t0;
+  a.Lq = Lq;
+  a.scale_log2 = p.scale * 1.4426950408889634f;
+  return launch_sparse_mla(tq, tkv, a, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_version(void) { return 1; }
+
+const char *dsa_status_string(dsa_status_t s) {
+  switch (s) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG: bad pointer, size or shape";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED: valid but unsupported shape or type";
+    case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE: workspace missing or too small";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA: a CUDA call failed";
+    case DSA_ERR_INTERNAL: return "DSA_ERR_INTERNAL: device status word reports a failure";
+  }
+  return "unknown dsa_status_t";
+}
+
+size_t dsa_indexer_topk_workspace(int L, int N, int H_I, int D_I, int topk, dsa_dtype_t dtype) {
+  if (L <= 0 || N <= 0 || H_I <= 0 || D_I <= 0 || topk <= 0) return 0;
+  (void)dtype;
+  const int QB = std::min(L, kDefaultQueryBlock);
+  return idx_fixed_bytes(QB, N) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
+}
+
+dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype, int L,
+                              int N, int H_I, int D_I, int q_pos0, int topk, int32_t *topk_idx, float *topk_score,
+                              void *workspace, size_t workspace_bytes, dsa_stream_t stream_) {
+  if (dtype != DSA_BF16 && dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID_ARG;
+  IndexerProblem p{q_idx, k_idx, w, dtype == DSA_FP8_E4M3, L, N, H_I, D_I, q_pos0, topk, topk_idx, topk_score};
+  dsa_status_t st = check_indexer_args(p);
+  if (st != DSA_OK) return st;
+  const int QB = std::min(L, kDefaultQueryBlock);
+  IdxWorkspace ws;
+  if (!carve_idx_ws(workspace, workspace_bytes, QB, N, &ws)) return DSA_ERR_WORKSPACE;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  CUtensorMap tq, tk;
+  if (!make_indexer_maps(p, &tq, &tk)) return DSA_ERR_CUDA;
+  if (cudaMemsetAsync(ws.status, 0, kHeaderBytes, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  for (int t0 = 0; t0 < L; t0 += QB) {
+    st = run_indexer_block(p, tq, tk, ws, t0, std::min(QB, L - t0), stream);
+    if (st != DSA_OK) return st;
+  }
+  return DSA_OK;
+}
+
+size_t dsa_sparse_mla_workspace(int L, int H, int topk) {
+  if (L <= 0 || H <= 0 || topk <= 0) return 0;
+  return kHeaderBytes;
+}
+
+dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, const int32_t *topk_idx, int L, int N, int H,
+                                    int topk, float scale, void *out, float *lse, void *workspace,
+                                    size_t workspace_bytes, dsa_stream_t stream_) {
+  MlaProblem p{q, kv, topk_idx, L, N, H, topk, scale, out, lse};
+  dsa_status_t st = check_mla_args(p);
+  if (st != DSA_OK) return st;
+  if (workspace == nullptr || workspace_bytes < kHeaderBytes) return DSA_ERR_WORKSPACE;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  CUtensorMap tq, tkv;
+  if (!make_mla_maps(p, &tq, &tkv)) return DSA_ERR_CUDA;
+  unsigned *status = static_cast<unsigned *>(workspace);
+  if (cudaMemsetAsync(status, 0, kHeaderBytes, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  return run_mla_block(p, tq, tkv, status, 0, L, stream);
+}
+
+size_t dsa_prefill_chunk_workspace(int L, int N, int H_I, int D_I, int H, int topk, int query_block,
+                                   dsa_dtype_t dtype, int want_topk_out) {
+  if (L <= 0 || N <= 0 || H_I <= 0 || D_I <= 0 || H <= 0 || topk <= 0) return 0;
+  (void)dtype;
+  const int QB = std::min(L, query_block > 0 ? query_block : kDefaultQueryBlock);
+  size_t bytes = idx_fixed_bytes(QB, N) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
+  if (!want_topk_out) bytes += align256(static_cast<size_t>(QB) * topk * 4);
+  return bytes;
+}
+
+}  // extern "C"
+
+namespace {
+
+dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
+                                const void *q, const void *kv, int L, int N, int H_I, int D_I, int H, int q_pos0,
+                                int topk, float scale, int query_block, int32_t *topk_idx_out, void *out, float *lse,
+                                void *workspace, size_t workspace_bytes, dsa_stream_t stream_, cudaEvent_t *events,
+                                int n_events) {
+  if (dtype != DSA_BF16 && dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID_ARG;
+  if (L <= 0 || topk <= 0) return DSA_ERR_INVALID_ARG;
+  const int QB = std::min(L, query_block > 0 ? query_block : kDefaultQueryBlock);
+  // Selected keys: the caller's buffer, or a block-sized region at the end of the workspace.
+  size_t idx_bytes = workspace_bytes;
+  int32_t *block_idx = nullptr;
+  if (topk_idx_out == nullptr) {
+    const size_t need = align256(static_cast<size_t>(QB) * topk * 4);
+    if (workspace == nullptr || workspace_bytes < need) return DSA_ERR_WORKSPACE;
+    idx_bytes = (workspace_bytes - need) & ~static_cast<size_t>(255);
+    block_idx = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + idx_bytes);
+  }
+  IndexerProblem ip{q_idx, k_idx, w, dtype == DSA_FP8_E4M3, L, N, H_I, D_I, q_pos0, topk,
+                    topk_idx_out ? topk_idx_out : block_idx, nullptr};
+  dsa_status_t st = check_indexer_args(ip);
+  if (st != DSA_OK) return st;
+  MlaProblem mp{q, kv, ip.topk_idx, L, N, H, topk, scale, out, lse};
+  st = check_mla_args(mp);
+  if (st != DSA_OK) return st;
+  IdxWorkspace ws;
+  if (!carve_idx_ws(workspace, idx_bytes, QB, N, &ws)) return DSA_ERR_WORKSPACE;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  CUtensorMap tq, tk, mq, mkv;
+  if (!make_indexer_maps(ip, &tq, &tk) || !make_mla_maps(mp, &mq, &mkv)) return DSA_ERR_CUDA;
+  const int nblocks = (L + QB - 1) / QB;
+  if (events != nullptr && n_events < 7 * nblocks) return DSA_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(ws.status, 0, kHeaderBytes, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  for (int t0 = 0; t0 < L; t0 += QB) {
+    const int Lb = std::min(QB, L - t0);
+    cudaEvent_t *ev = events ? events + 7 * (t0 / QB) : nullptr;
+    IndexerProblem bp = ip;
+    MlaProblem bm = mp;
+    if (block_idx != nullptr) {
+      // The block's indices land at rows [0, Lb) of the workspace buffer.
+      bp.topk_idx = block_idx - static_cast<long long>(t0) * topk;
+      bm.topk_idx = bp.topk_idx;
+    }
+    st = run_indexer_block(bp, tq, tk, ws, t0, Lb, stream, ev);
+    if (st != DSA_OK) return st;
+    st = run_mla_block(bm, mq, mkv, ws.status, t0, Lb, stream);
+    if (st != DSA_OK) return st;
+    if (!mark(ev, 6, stream)) return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dsa_status_t dsa_prefill_chunk(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
+                               const void *q, const void *kv, int L, int N, int H_I, int D_I, int H, int q_pos0,
+                               int topk, float scale, int query_block, int32_t *topk_idx_out, void *out, float *lse,
+                               void *workspace, size_t workspace_bytes, dsa_stream_t stream) {
+  return prefill_chunk_impl(q_idx, k_idx, w, dtype, q, kv, L, N, H_I, D_I, H, q_pos0, topk, scale, query_block,
+                            topk_idx_out, out, lse, workspace, workspace_bytes, stream, nullptr, 0);
+}
+
+dsa_status_t dsa_prefill_chunk_profiled(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
+                                        const void *q, const void *kv, int L, int N, int H_I, int D_I, int H,
+                                        int q_pos0, int topk, float scale, int query_block, int32_t *topk_idx_out,
+                                        void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                        dsa_stream_t stream, void *const *events, int n_events) {
+  if (events == nullptr) return DSA_ERR_INVALID_ARG;
+  return prefill_chunk_impl(q_idx, k_idx, w, dtype, q, kv, L, N, H_I, D_I, H, q_pos0, topk, scale, query_block,
+                            topk_idx_out, out, lse, workspace, workspace_bytes, stream,
+                            reinterpret_cast<cudaEvent_t *>(const_cast<void **>(events)), n_events);
+}
+
+dsa_status_t dsa_workspace_status(const void *workspace, dsa_stream_t stream_, unsigned *flags) {
+  if (workspace == nullptr || flags == nullptr) return DSA_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  unsigned v = 0;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemcpy(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+  *flags = v;
+  return v == 0 ? DSA_OK : DSA_ERR_INTERNAL;
+}
+
+}  // extern "C"

@@ -1,0 +1,71 @@
+// dsa_internal.h -- declarations shared by the library's translation units
+// (kernel argument blocks and launchers).  Not part of the public C ABI.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace dsa {
+
+// Arguments of one indexer launch (one query block).
+struct IndexerArgs {
+  const float *w;                 // [Lb, H_I] head weights of the block's queries
+  const unsigned *tau;            // [Lb] threshold score keys (EMIT mode; 0 = keep all)
+  float *dense;                   // [Lb, dense_ld] sample scores (PILOT mode)
+  unsigned long long *cand;       // [Lb, cap] candidate keys (EMIT mode)
+  int *cand_count;                // [Lb] candidates seen (may exceed cap)
+  unsigned *status;               // device status word
+  int dense_ld;
+  int cap;
+  int Lb;                         // queries in the block
+  int q_pos0;                     // position of the block's first query
+  int n_keys;                     // rows of the key tensor map (PILOT: samples, EMIT: N)
+  int q_row0;                     // first row of the block in the [L*H_I, D_I] query tensor map
+  int total_tiles;                // sum over query groups of their 128-key tiles
+  int pilot;                      // 1 = PILOT mode
+};
+
+cudaError_t launch_indexer(const CUtensorMap &tq, const CUtensorMap &tk, const IndexerArgs &a, int D_I, int H_I,
+                           bool fp8, bool pilot, int grid, cudaStream_t stream);
+bool indexer_supported(int D_I, int H_I, bool fp8);
+int indexer_queries_per_group(int H_I);
+
+// Threshold / selection / fallback stage.
+struct SelectArgs {
+  const void *q_idx;              // [L, H_I, D_I] whole chunk (fallback rescoring)
+  const void *k_idx;              // [N, D_I]
+  const float *w;                 // [L, H_I] whole chunk
+  const float *dense;             // [Lb, dense_ld] pilot sample scores, or nullptr
+  unsigned *tau;                  // [Lb] threshold score keys
+  const unsigned long long *cand; // [Lb, cap]
+  int *cand_count;                // [Lb]
+  int *fb_list;                   // [Lb] queries that need the exact fallback
+  int *fb_counters;               // [0] = count, [1] = next
+  float *fb_scratch;              // [fb_slots, N] fallback score rows
+  unsigned *status;
+  int32_t *topk_idx;              // [L, topk] whole chunk
+  float *topk_score;              // [L, topk] or nullptr
+  int dense_ld, n_samples, cap, fb_slots;
+  int t0, Lb, q_pos0;             // block: first query (chunk row), size, position of first query
+  int N, H_I, D_I, topk, fp8;
+};
+
+cudaError_t launch_threshold(const SelectArgs &a, cudaStream_t stream);
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream);
+cudaError_t launch_fallback(const SelectArgs &a, cudaStream_t stream);
+
+// Sparse absorbed-MLA attention.
+struct MlaArgs {
+  const int32_t *topk_idx;        // [L, topk]
+  uint16_t *out;                  // [L, H, 512] bf16 bits
+  float *lse;                     // [L, H] or nullptr
+  unsigned *status;
+  int L, N, H, topk;
+  int t0, Lq;                     // queries [t0, t0 + Lq) of the chunk in this launch
+  float scale_log2;               // softmax scale * log2(e)
+};
+
+cudaError_t launch_sparse_mla(const CUtensorMap &tq, const CUtensorMap &tkv, const MlaArgs &a, cudaStream_t stream);
+
+}  // namespace dsa

@@ -1,0 +1,396 @@
+// indexer.cu -- lightning-indexer scoring on the 5th-generation tensor cores.
+//
+// For one block of queries the kernel computes, for every (query t, visible
+// key s) pair,
+//     I[t,s] = sum_h w[t,h] * max(0, q_idx[t,h,:] . k_idx[s,:])
+// (the DeepSeek Sparse Attention lightning indexer: 32 ReLU-gated, weighted
+// heads over one shared indexer key per position; mlx-lm PR #1997 "GLM prefill
+// now attends only to the keys its indexer picks", section "How it works"),
+// and never writes the L x N score matrix: the ReLU / head-weight reduction is
+// fused into the accumulator epilogue and each score is either
+//   * PILOT mode: written densely for a strided sample of the keys (the small
+//     sample that LiteTopK, arXiv 2607.11976 Abstract, uses to estimate each
+//     query's score range), or
+//   * EMIT mode: compared with the query's threshold and, when it passes,
+//     appended to that query's candidate list ("write back only promising
+//     candidates", LiteTopK Abstract).
+//
+// Tile shape (swap-AB): A = 128 keys x D_I (UMMA M = 128), B = a group of
+// 256 / H_I queries x H_I heads = 256 rows x D_I (UMMA N = 256), K = D_I.
+// Each TMEM lane then holds one key and each epilogue thread reduces the heads
+// of its key locally.  Warp roles: warp 0 TMA producer, warp 1 MMA issuer and
+// TMEM owner, warps 2..9 epilogue (two per TMEM lane quarter, each pair
+// splitting the 256 accumulator columns).  The accumulator is double-buffered
+// (2 x 256 columns) so the epilogue of tile i overlaps the MMA of tile i+1.
+#include <cuda_runtime.h>
+
+#include "dsa_internal.h"
+#include "ptx.cuh"
+
+namespace dsa {
+
+template <int DI, int HI, bool FP8>
+struct IdxCfg {
+  static constexpr int ESZ = FP8 ? 1 : 2;
+  static constexpr int ROW_BYTES = DI * ESZ;
+  static constexpr int ATOMS = ROW_BYTES / 128;  // 128-byte swizzle atoms along K
+  static constexpr int ATOM_ELEMS = 128 / ESZ;
+  static constexpr int KSTEP = FP8 ? 32 : 16;  // K of one tcgen05.mma
+  static constexpr int KSTEPS_PER_ATOM = ATOM_ELEMS / KSTEP;
+  static constexpr int BM = 128;  // keys per tile
+  static constexpr int BN = 256;  // query-head rows per group
+  static constexpr int QG = BN / HI;
+  static constexpr int K_TILE = BM * ROW_BYTES;
+  static constexpr int Q_TILE = BN * ROW_BYTES;
+  static constexpr int STAGES = (K_TILE <= 16384) ? 8 : 4;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = 64 + EPI_WARPS * 32;
+  // shared memory carve-up (offsets from a 1024-aligned base)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_TILE;
+  static constexpr int OFF_W = OFF_K + STAGES * K_TILE;       // [EPI_WARPS][128] floats
+  static constexpr int OFF_TAU = OFF_W + EPI_WARPS * 128 * 4;  // [EPI_WARPS][QG/2] floats
+  static constexpr int OFF_BAR = OFF_TAU + EPI_WARPS * 128 * 4;  // mbarriers
+  static constexpr int NBAR = 2 * STAGES + 2 + 4 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // tmem addr, abort flag, counters
+  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
+  static_assert(ROW_BYTES % 128 == 0, "indexer rows must be whole 128-byte atoms");
+  static_assert(QG * HI == BN, "H_I must divide 256");
+  static_assert((QG / 2) * HI == 128, "each epilogue half covers 128 columns");
+};
+
+// Per-group number of 128-key tiles.
+__device__ __forceinline__ int idx_group_tiles(const IndexerArgs &a, int g, int QG) {
+  int keys;
+  if (a.pilot) {
+    keys = a.n_keys;
+  } else {
+    int last = min(a.Lb, (g + 1) * QG);  // queries [g*QG, last) ; positions up to q_pos0 + last - 1
+    keys = min(a.n_keys, a.q_pos0 + last);
+  }
+  return (keys + 127) / 128;
+}
+
+// Tile range of this CTA in the linearised (group, key tile) space.
+struct TileCursor {
+  int g, tile, ntiles_g, left;
+};
+
+__device__ __forceinline__ TileCursor idx_cursor_begin(const IndexerArgs &a, int QG) {
+  const long long T = a.total_tiles;
+  const long long u0 = T * blockIdx.x / gridDim.x;
+  const long long u1 = T * (blockIdx.x + 1) / gridDim.x;
+  TileCursor c;
+  c.left = static_cast<int>(u1 - u0);
+  long long acc = 0;
+  int g = 0;
+  int nt = idx_group_tiles(a, 0, QG);
+  while (acc + nt <= u0) {
+    acc += nt;
+    ++g;
+    nt = idx_group_tiles(a, g, QG);
+  }
+  c.g = g;
+  c.tile = static_cast<int>(u0 - acc);
+  c.ntiles_g = nt;
+  return c;
+}
+
+__device__ __forceinline__ void idx_cursor_next(TileCursor &c, const IndexerArgs &a, int QG) {
+  --c.left;
+  if (++c.tile == c.ntiles_g) {
+    c.tile = 0;
+    ++c.g;
+    c.ntiles_g = idx_group_tiles(a, c.g, QG);
+  }
+}
+
+template <int DI, int HI, bool FP8, bool PILOT>
+__global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                   IndexerArgs a) {
+  using C = IdxCfg<DI, HI, FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *q_s = smem + C::OFF_Q;
+  uint8_t *k_s = smem + C::OFF_K;
+  float *w_s = reinterpret_cast<float *>(smem + C::OFF_W);
+  float *tau_s = reinterpret_cast<float *>(smem + C::OFF_TAU);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+  uint64_t *full = bars;                    // [STAGES] TMA -> MMA
+  uint64_t *empty = bars + C::STAGES;       // [STAGES] MMA -> TMA
+  uint64_t *q_full = bars + 2 * C::STAGES;  // query tile landed
+  uint64_t *q_empty = q_full + 1;           // MMA done with the query tile
+  uint64_t *acc_full = q_full + 2;          // [2] MMA -> epilogue
+  uint64_t *acc_empty = q_full + 4;         // [2] epilogue -> MMA
+  uint64_t *drain = q_full + 6;             // MMA drain on abort
+  unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + C::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
+  int *consumed = reinterpret_cast<int *>(smem + C::OFF_MISC + 16);  // k tiles the MMA warp consumed
+  int *q_consumed = reinterpret_cast<int *>(smem + C::OFF_MISC + 20);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], C::EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *consumed = 0;
+    *q_consumed = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmap_q);
+    prefetch_tensormap(&tmap_k);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const unsigned tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      TileCursor c = idx_cursor_begin(a, C::QG);
+      int stage = 0;
+      unsigned phase = 0, qphase = 0;
+      int prev_g = -1, issued = 0, q_issued = 0;
+      bool ok = true;
+      while (c.left > 0) {
+        if (c.g != prev_g) {
+          if (prev_g >= 0) {
+            if (!mbar_wait(q_empty, qphase, abort_flag)) { ok = false; break; }
+            qphase ^= 1u;
+          }
+          mbar_arrive_expect_tx(q_full, C::Q_TILE);
+          for (int at = 0; at < C::ATOMS; ++at)
+            tma_load_2d(q_s + at * C::BN * 128, &tmap_q, q_full, at * C::ATOM_ELEMS, a.q_row0 + c.g * C::BN);
+          ++q_issued;
+          prev_g = c.g;
+        }
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&full[stage], C::K_TILE);
+        for (int at = 0; at < C::ATOMS; ++at)
+          tma_load_2d(k_s + stage * C::K_TILE + at * C::BM * 128, &tmap_k, &full[stage], at * C::ATOM_ELEMS,
+                      c.tile * C::BM);
+        ++issued;
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        idx_cursor_next(c, a, C::QG);
+      }
+      if (!ok) {
+        atomicOr(a.status, DEV_TIMEOUT);
+        *abort_flag = 1;
+      }
+      // Never leave with copies in flight: wait for every issued load to land.
+      const int done = *reinterpret_cast<volatile int *>(consumed);
+      for (int i = done; i < issued; ++i) mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1u, nullptr);
+      if (q_issued > *reinterpret_cast<volatile int *>(q_consumed))
+        mbar_wait(q_full, static_cast<unsigned>(q_issued - 1) & 1u, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    TileCursor c = idx_cursor_begin(a, C::QG);
+    constexpr unsigned idesc = make_idesc(C::BM, C::BN, FP8 ? 0u : 1u, 0u, 0u);
+    int stage = 0, acc = 0, prev_g = -1, n = 0;
+    unsigned phase = 0, acc_phase = 0, qphase = 0;
+    bool ok = true;
+    while (c.left > 0) {
+      const int g = c.g;
+      if (g != prev_g) {
+        if (!mbar_wait(q_full, qphase, abort_flag)) { ok = false; break; }
+        qphase ^= 1u;
+        prev_g = g;
+        if (lane == 0) *reinterpret_cast<volatile int *>(q_consumed) += 1;
+      }
+      if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      TileCursor nx = c;
+      idx_cursor_next(nx, a, C::QG);
+      const bool last_of_group = (nx.left == 0) || (nx.g != g);
+      if (lane == 0) {
+        const unsigned d_tmem = tmem_base + acc * 256;
+        const unsigned a_base = smem_u32(k_s + stage * C::K_TILE);
+        const unsigned b_base = smem_u32(q_s);
+#pragma unroll
+        for (int at = 0; at < C::ATOMS; ++at) {
+#pragma unroll
+          for (int ks = 0; ks < C::KSTEPS_PER_ATOM; ++ks) {
+            const uint64_t ad = smem_desc_sw128(a_base + at * C::BM * 128 + ks * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(b_base + at * C::BN * 128 + ks * 32, 16, 1024);
+            const unsigned accum = (at | ks) ? 1u : 0u;
+            if (FP8)
+              mma_fp8_ss(d_tmem, ad, bd, idesc, accum);
+            else
+              mma_bf16_ss(d_tmem, ad, bd, idesc, accum);
+          }
+        }
+        tc_commit(&empty[stage]);
+        tc_commit(&acc_full[acc]);
+        if (last_of_group) tc_commit(q_empty);
+      }
+      __syncwarp();
+      ++n;
+      if (lane == 0) *reinterpret_cast<volatile int *>(consumed) = n;
+      if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      c = nx;
+    }
+    if (!ok && lane == 0) {
+      atomicOr(a.status, DEV_TIMEOUT);
+      *abort_flag = 1;
+    }
+    // Drain: every MMA this warp issued must finish before TMEM is released.
+    if (lane == 0) {
+      tc_commit(drain);
+      mbar_wait(drain, 0u, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;          // 0..7
+    const int quarter = warp & 3;     // TMEM lane quarter this warp may access
+    const int half = ew >> 2;         // which 128 accumulator columns
+    constexpr int QH = C::QG / 2;     // queries per half
+    TileCursor c = idx_cursor_begin(a, C::QG);
+    int acc = 0, prev_g = -1;
+    unsigned acc_phase = 0;
+    bool ok = true;
+    const unsigned lane_mask_lt = (1u << lane) - 1u;
+    float *w_w = w_s + ew * 128;   // this warp's head weights: [QH queries][HI]
+    unsigned *tau_w = reinterpret_cast<unsigned *>(tau_s) + ew * 128;
+    while (c.left > 0) {
+      const int g = c.g;
+      if (g != prev_g) {
+        // Each warp stages the head weights / thresholds of its own queries
+        // (no cross-warp barrier, so an aborting warp cannot strand the others).
+        __syncwarp();
+        for (int j = lane; j < 128; j += 32) {
+          const int tl = g * C::QG + half * QH + j / HI;
+          w_w[j] = (tl < a.Lb) ? a.w[static_cast<long long>(g * C::QG + half * QH) * HI + j] : 0.0f;
+        }
+        if (!PILOT) {
+          for (int j = lane; j < QH; j += 32) {
+            const int tl = g * C::QG + half * QH + j;
+            tau_w[j] = (tl < a.Lb) ? a.tau[tl] : 0xFFFFFFFFu;
+          }
+        }
+        __syncwarp();
+        prev_g = g;
+      }
+      if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t v[4][32];
+      const unsigned taddr = tmem_base + (static_cast<unsigned>(quarter * 32) << 16) + acc * 256 + half * 128;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_ld_32x32b_x32(taddr + ch * 32, v[ch]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+
+      const int key = c.tile * C::BM + quarter * 32 + lane;
+#pragma unroll
+      for (int qq = 0; qq < QH; ++qq) {
+        const int qg = half * QH + qq;  // query within the group
+        const int tl = g * C::QG + qg;  // query within the block
+        float score = 0.0f;
+#pragma unroll
+        for (int h = 0; h < HI; ++h) {
+          const int col = qq * HI + h;
+          const float s = __uint_as_float(v[col / 32][col % 32]);
+          score = fmaf(w_w[qq * HI + h], fmaxf(s, 0.0f), score);
+        }
+        if (PILOT) {
+          if (tl < a.Lb && key < a.n_keys) a.dense[static_cast<long long>(tl) * a.dense_ld + key] = score;
+        } else {
+          const bool pass = (tl < a.Lb) && (key <= a.q_pos0 + tl) && (float_order_key(score) >= tau_w[qq]);
+          const unsigned m = __ballot_sync(0xffffffffu, pass);
+          if (m) {
+            const int leader = __ffs(m) - 1;
+            int base = 0;
+            if (lane == leader) base = atomicAdd(&a.cand_count[tl], __popc(m));
+            base = __shfl_sync(0xffffffffu, base, leader);
+            if (pass) {
+              const int pos = base + __popc(m & lane_mask_lt);
+              if (pos < a.cap) {
+                const unsigned long long k64 = (static_cast<unsigned long long>(float_order_key(score)) << 32) |
+                                               static_cast<unsigned>(~static_cast<unsigned>(key));
+                a.cand[static_cast<long long>(tl) * a.cap + pos] = k64;
+              }
+            }
+          }
+        }
+      }
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      idx_cursor_next(c, a, C::QG);
+    }
+    if (!ok) {
+      if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int DI, int HI, bool FP8, bool PILOT>
+static cudaError_t launch_indexer_t(const CUtensorMap &tq, const CUtensorMap &tk, const IndexerArgs &a, int grid,
+                                    cudaStream_t stream) {
+  using C = IdxCfg<DI, HI, FP8>;
+  auto kern = indexer_kernel<DI, HI, FP8, PILOT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, a);
+  return cudaGetLastError();
+}
+
+int indexer_queries_per_group(int H_I) { return 256 / H_I; }
+
+cudaError_t launch_indexer(const CUtensorMap &tq, const CUtensorMap &tk, const IndexerArgs &a, int D_I, int H_I,
+                           bool fp8, bool pilot, int grid, cudaStream_t stream) {
+#define DSA_IDX_CASE(DI_, HI_, FP8_)                                                            \
+  if (D_I == DI_ && H_I == HI_ && fp8 == FP8_)                                                  \
+    return pilot ? launch_indexer_t<DI_, HI_, FP8_, true>(tq, tk, a, grid, stream)              \
+                 : launch_indexer_t<DI_, HI_, FP8_, false>(tq, tk, a, grid, stream);
+  DSA_IDX_CASE(128, 32, false)
+  DSA_IDX_CASE(128, 32, true)
+  DSA_IDX_CASE(64, 4, false)
+  DSA_IDX_CASE(128, 4, false)
+  DSA_IDX_CASE(64, 32, false)
+  DSA_IDX_CASE(128, 16, false)
+  DSA_IDX_CASE(128, 16, true)
+  DSA_IDX_CASE(128, 8, false)
+  DSA_IDX_CASE(128, 8, true)
+  DSA_IDX_CASE(128, 4, true)
+#undef DSA_IDX_CASE
+  return cudaErrorInvalidValue;
+}
+
+bool indexer_supported(int D_I, int H_I, bool fp8) {
+  if (fp8) return D_I == 128 && (H_I == 32 || H_I == 16 || H_I == 8 || H_I == 4);
+  if (D_I == 128) return H_I == 32 || H_I == 16 || H_I == 8 || H_I == 4;
+  if (D_I == 64) return H_I == 32 || H_I == 4;
+  return false;
+}
+
+}  // namespace dsa

@@ -1,0 +1,387 @@
+// mla.cu -- sparse absorbed-MLA attention over each query's selected keys.
+//
+// mlx-lm PR #1997 ("GLM prefill now attends only to the keys its indexer
+// picks", section "How it works"): the latent and rope caches are joined into
+// one 576-wide key per position, the top-k rows a query picked are gathered
+// once and shared by all its heads, and attention runs in the absorbed latent
+// space, so a chunk costs L * top-k instead of L * N.  For query t and head h:
+//     z_j = scale * (q_lat[t,h] . kv_lat[i_j] + q_rope[t,h] . k_rope[i_j])
+//     out[t,h] = sum_j softmax(z)_j * kv_lat[i_j]          (512 wide)
+// Index -1 marks a skipped entry (llama.cpp PR #25917, discussion).
+//
+// B200 mapping.  One CTA per (query, group of 64 heads).  Per 64-key tile:
+//   * TMA tile::gather4 loads the 64 selected rows (9 column atoms of 128 B,
+//     128-byte swizzle) straight into the UMMA operand layout;
+//   * S = Q K^T on tcgen05 (M = 64 heads, N = 64 keys, K = 576), fp32 in TMEM;
+//   * softmax warps read S from TMEM, keep a running max (rescaling the output
+//     only when the max grows by more than 2^8) and write P (bf16) to shared
+//     memory in the UMMA layout;
+//   * O += P V on tcgen05 (M = 64, N = 2 x 256 latent columns, K = 64 keys),
+//     V read in place from the gathered tile as an MN-major operand.
+// TMEM: the two 64 x 256 fp32 halves of O sit in the two half-subpartitions
+// (lanes 0-15 and 16-31 of each 32-lane quarter) of columns 0-255, the two S
+// buffers in columns 256-383.  Warp roles: warp 0 gather producer, warp 1 MMA
+// issuer / TMEM owner, warps 2-5 softmax and output.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "dsa_internal.h"
+#include "ptx.cuh"
+
+namespace dsa {
+namespace mla {
+
+constexpr int HT = 64;           // heads per CTA (UMMA M)
+constexpr int BK = 64;           // keys per tile
+constexpr int DIM = 576;         // joined key width
+constexpr int LAT = 512;         // value width
+constexpr int ATOMS = DIM / 64;  // 128-byte column atoms
+constexpr int ATOM_BYTES = 64 * 128;  // 64 rows x 128 B
+constexpr int Q_BYTES = ATOMS * ATOM_BYTES;
+constexpr int KV_BYTES = ATOMS * ATOM_BYTES;
+constexpr int P_BYTES = HT * BK * 2;
+constexpr int STAGES = 2;
+constexpr int THREADS = 192;
+constexpr int OFF_Q = 0;
+constexpr int OFF_KV = OFF_Q + Q_BYTES;
+constexpr int OFF_P = OFF_KV + STAGES * KV_BYTES;
+constexpr int OFF_BAR = OFF_P + P_BYTES;
+constexpr int NBAR = 1 + 2 * STAGES + 4 + 2 + 1;
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
+constexpr float kRescaleLog2 = 8.0f;
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_kv,
+                      MlaArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *q_s = smem + OFF_Q;
+  uint8_t *kv_s = smem + OFF_KV;
+  uint8_t *p_s = smem + OFF_P;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  uint64_t *q_full = bars;
+  uint64_t *kv_full = bars + 1;           // [2]
+  uint64_t *kv_empty = bars + 3;          // [2]
+  uint64_t *s_full = bars + 5;            // [2]
+  uint64_t *s_free = bars + 7;            // [2]
+  uint64_t *p_full = bars + 9;
+  uint64_t *p_free = bars + 10;
+  uint64_t *drain = bars + 11;
+  unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+  unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + OFF_MISC + 8);  // [2]
+  int *consumed = reinterpret_cast<int *>(smem + OFF_MISC + 24);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int t = a.t0 + blockIdx.x;
+  const int hg = blockIdx.y;
+  const int ntiles = (a.topk + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(p_free, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *consumed = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmap_q);
+    prefetch_tensormap(&tmap_kv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const unsigned tmem = *tmem_slot;
+  const unsigned o_lo = tmem;                          // lanes 0-15 of each quarter, cols 0-255
+  const unsigned o_hi = tmem + (16u << 16);            // lanes 16-31 of each quarter, cols 0-255
+  const unsigned s_col = tmem + 256;                   // S buffers: cols 256-319, 320-383
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ gather producer
+    bool ok = true;
+    int issued = 0;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, Q_BYTES);
+      const int row0 = t * a.H + hg * HT;
+      for (int at = 0; at < ATOMS; ++at) tma_load_2d(q_s + at * ATOM_BYTES, &tmap_q, q_full, at * 64, row0);
+    }
+    const int32_t *idx_row = a.topk_idx + static_cast<long long>(t) * a.topk;
+    for (int j = 0; j < ntiles; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1u, abort_flag)) { ok = false; break; }
+      int r[4];
+      unsigned bits = 0;
+      if (lane < 16) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int pos = j * BK + lane * 4 + e;
+          const int v = pos < a.topk ? idx_row[pos] : -1;
+          const bool good = v >= 0 && v < a.N;
+          if (v >= a.N || v < -1) atomicOr(a.status, DEV_BAD_INDEX);
+          r[e] = good ? v : 0;
+          bits |= (good ? 1u : 0u) << e;
+        }
+      }
+      // 64-bit validity mask of this tile: lane l contributes bits 4l..4l+3.
+      unsigned lo = (lane < 8) ? (bits << (4 * lane)) : 0u;
+      unsigned hi = (lane >= 8 && lane < 16) ? (bits << (4 * (lane - 8))) : 0u;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        lo |= __shfl_xor_sync(0xffffffffu, lo, off);
+        hi |= __shfl_xor_sync(0xffffffffu, hi, off);
+      }
+      if (lane == 0) {
+        valid_s[st] = (static_cast<unsigned long long>(hi) << 32) | lo;
+        mbar_arrive_expect_tx(&kv_full[st], KV_BYTES);
+      }
+      __syncwarp();
+      if (lane < 16) {
+        uint8_t *dst = kv_s + st * KV_BYTES + lane * 4 * 128;
+#pragma unroll
+        for (int at = 0; at < ATOMS; ++at)
+          tma_gather4(dst + at * ATOM_BYTES, &tmap_kv, &kv_full[st], at * 64, r[0], r[1], r[2], r[3]);
+      }
+      ++issued;
+    }
+    if (!ok) {
+      if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
+      *abort_flag = 1;
+    }
+    if (lane == 0) {
+      // Never leave with copies in flight.
+      mbar_wait(q_full, 0u, nullptr);
+      const int done = *reinterpret_cast<volatile int *>(consumed);
+      for (int i = done; i < issued; ++i) mbar_wait(&kv_full[i & 1], (i >> 1) & 1u, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr unsigned idesc_qk = make_idesc(HT, BK, 1u, 0u, 0u);   // S = Q K^T, both K-major
+    constexpr unsigned idesc_pv = make_idesc(HT, 256, 1u, 0u, 1u);  // O += P V, V MN-major
+    bool ok = mbar_wait(q_full, 0u, abort_flag);
+    const unsigned q_base = smem_u32(q_s);
+    const unsigned p_base = smem_u32(p_s);
+    auto issue_pv = [&](int jj) {
+      const unsigned v_base = smem_u32(kv_s + (jj & 1) * KV_BYTES);
+#pragma unroll
+      for (int ks = 0; ks < BK / 16; ++ks) {
+        const uint64_t pd = smem_desc_sw128(p_base + ks * 32, 16, 1024);
+        const uint64_t vlo = smem_desc_sw128(v_base + ks * 2048, ATOM_BYTES, 1024);
+        const uint64_t vhi = smem_desc_sw128(v_base + 4 * ATOM_BYTES + ks * 2048, ATOM_BYTES, 1024);
+        const unsigned acc = (jj > 0 || ks > 0) ? 1u : 0u;
+        mma_bf16_ss(o_lo, pd, vlo, idesc_pv, acc);
+        mma_bf16_ss(o_hi, pd, vhi, idesc_pv, acc);
+      }
+      tc_commit(&kv_empty[jj & 1]);
+      tc_commit(p_free);
+    };
+    for (int j = 0; ok && j < ntiles; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(&kv_full[st], (j >> 1) & 1u, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&s_free[st], ((j >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      if (lane == 0) {
+        const unsigned k_base = smem_u32(kv_s + st * KV_BYTES);
+        for (int at = 0; at < ATOMS; ++at) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t qd = smem_desc_sw128(q_base + at * ATOM_BYTES + ks * 32, 16, 1024);
+            const uint64_t kd = smem_desc_sw128(k_base + at * ATOM_BYTES + ks * 32, 16, 1024);
+            mma_bf16_ss(s_col + st * 64, qd, kd, idesc_qk, (at | ks) ? 1u : 0u);
+          }
+        }
+        tc_commit(&s_full[st]);
+        *reinterpret_cast<volatile int *>(consumed) = j + 1;
+      }
+      __syncwarp();
+      if (j > 0) {
+        if (!mbar_wait(p_full, (j - 1) & 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) issue_pv(j - 1);
+        __syncwarp();
+      }
+    }
+    if (ok) {
+      if (mbar_wait(p_full, (ntiles - 1) & 1u, abort_flag)) {
+        tc_fence_after();
+        if (lane == 0) issue_pv(ntiles - 1);
+        __syncwarp();
+      } else {
+        ok = false;
+      }
+    }
+    if (!ok) {
+      if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
+      *abort_flag = 1;
+    }
+    if (lane == 0) {
+      tc_commit(drain);
+      mbar_wait(drain, 0u, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax + output
+    const int quarter = warp & 3;
+    const int r16 = lane & 15;
+    const int row = quarter * 16 + r16;  // head within the CTA's group
+    const unsigned lane_base = static_cast<unsigned>(quarter * 32) << 16;
+    float m_used = -INFINITY, l = 0.0f, l_exact = 0.0f;  // l: sum of the bf16 P used; l_exact: fp32 sum for the LSE
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int sb = j & 1;
+      if (!mbar_wait(&s_full[sb], (j >> 1) & 1u, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[2][32];
+      tmem_ld_32x32b_x32(s_col + lane_base + sb * 64, sv[0]);
+      tmem_ld_32x32b_x32(s_col + lane_base + sb * 64 + 32, sv[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[sb]);
+      const unsigned long long vmask = valid_s[j & 1];
+      float z[64];
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const bool v = (vmask >> c) & 1ull;
+        z[c] = v ? __uint_as_float(sv[c >> 5][c & 31]) * a.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, z[c]);
+      }
+      const float m_old = m_used;
+      bool rescale = false;
+      if (tmax > m_used + kRescaleLog2 || (m_used == -INFINITY && tmax > -INFINITY)) {
+        rescale = (m_used != -INFINITY) && (j > 0);
+        m_used = tmax;
+      }
+      // P in bf16, rounded once; the normaliser sums the rounded values.
+      uint32_t pk[32];
+      float tsum = 0.0f, tsum_exact = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        const float p0 = (m_used == -INFINITY) ? 0.0f : fast_exp2(z[c] - m_used);
+        const float p1 = (m_used == -INFINITY) ? 0.0f : fast_exp2(z[c + 1] - m_used);
+        const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
+        const float2 br = __bfloat1622float2(b);
+        tsum += br.x + br.y;
+        tsum_exact += p0 + p1;
+        pk[c >> 1] = *reinterpret_cast<const uint32_t *>(&b);
+      }
+      const float alpha = rescale ? fast_exp2(m_old - m_used) : 1.0f;
+      l = l * alpha + tsum;
+      l_exact = l_exact * alpha + tsum_exact;
+      if (j > 0) {
+        if (!mbar_wait(p_free, (j - 1) & 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+      }
+      // Rescale O (both halves) when the running max moved: lanes 0-15 own the
+      // O_lo rows, lanes 16-31 the O_hi rows of the same heads.
+      const bool any_rescale = __any_sync(0xffffffffu, rescale && lane < 16);
+      if (any_rescale) {
+        const float my_alpha = __shfl_sync(0xffffffffu, alpha, r16);
+        const bool mine = __shfl_sync(0xffffffffu, rescale ? 1 : 0, r16) != 0;
+        // One 32x32b access covers lanes 32q..32q+31: O_lo rows then O_hi rows.
+        const unsigned obase = o_lo + lane_base;
+#pragma unroll 1
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t ov[32];
+          tmem_ld_32x32b_x32(obase + ch * 32, ov);
+          tmem_ld_wait();
+          if (mine) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * my_alpha);
+          }
+          tmem_st_32x32b_x32(obase + ch * 32, ov);
+        }
+        tmem_st_wait();
+      }
+      if (lane < 16) {
+        uint8_t *prow = p_s + row * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 v = make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+          *reinterpret_cast<uint4 *>(prow + ((ch ^ (row & 7)) << 4)) = v;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok) ok = mbar_wait(p_free, (ntiles - 1) & 1u, abort_flag);
+    if (!ok) {
+      if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
+      *abort_flag = 1;
+    } else {
+      tc_fence_after();
+      const float l_row = __shfl_sync(0xffffffffu, l, r16);
+      const float inv = l_row > 0.0f ? 1.0f / l_row : 0.0f;
+      const int head = hg * HT + row;
+      const int dim0 = lane < 16 ? 0 : 256;
+      uint16_t *orow = a.out + (static_cast<long long>(t) * a.H + head) * LAT + dim0;
+#pragma unroll 1
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t ov[32];
+        tmem_ld_32x32b_x32(o_lo + lane_base + ch * 32, ov);
+        tmem_ld_wait();
+        if (head < a.H) {
+          uint32_t pkd[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const __nv_bfloat162 b =
+                __floats2bfloat162_rn(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
+            pkd[e] = *reinterpret_cast<const uint32_t *>(&b);
+          }
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + ch * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+        }
+      }
+      if (lane < 16 && head < a.H && a.lse != nullptr) {
+        a.lse[static_cast<long long>(t) * a.H + head] =
+            l_exact > 0.0f ? (m_used + log2f(l_exact)) * 0.69314718055994530942f : -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace mla
+
+cudaError_t launch_sparse_mla(const CUtensorMap &tq, const CUtensorMap &tkv, const MlaArgs &a, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(mla::sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       mla::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.Lq, (a.H + mla::HT - 1) / mla::HT);
+  mla::sparse_mla_kernel<<<grid, mla::THREADS, mla::SMEM_BYTES, stream>>>(tq, tkv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

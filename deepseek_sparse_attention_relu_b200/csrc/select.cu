@@ -1,0 +1,304 @@
+// select.cu -- exact top-k selection from the indexer's pruned candidates.
+//
+// LiteTopK (arXiv 2607.11976, Abstract) keeps a tight approximate threshold
+// from a small sample, writes back only the candidates above it, and still
+// returns the exact top-k.  The B200 version here has three steps per query
+// block:
+//   1. threshold_kernel: from the indexer's dense scores of a strided key
+//      sample, pick the r-th best sample score as the query's threshold, with r
+//      chosen so that, by the order statistics of a uniform sample, at least
+//      topk visible keys lie above it with a 5-sigma margin.
+//   2. select_kernel: if the query's candidate list holds at least topk keys and
+//      did not overflow, it contains the exact top-k (every key scoring at
+//      least the threshold was written).  A block-wide MSB-first radix select on
+//      64-bit keys (order-preserving score bits << 32 | ~key index) finds the
+//      k-th best; the winners are emitted in ascending key order with -1
+//      padding (the int32 index-mask convention of llama.cpp PR #25917,
+//      discussion).  Equal scores go to the smaller index.
+//   3. fallback_kernel: any query the sample misjudged (too few or too many
+//      candidates) is rescored over all visible keys on the CUDA cores and
+//      selected exactly, so the result never depends on the sample.
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "dsa_internal.h"
+#include "ptx.cuh"
+
+namespace dsa {
+
+constexpr int kSelThreads = 512;
+constexpr int kMaxTopk = 4096;
+
+// Block-wide MSB-first radix select.  Among n unique keys (fetch(i), i < n) find
+// (prefix, mask) such that exactly `need` keys satisfy (key & mask) >= prefix,
+// i.e. key >= prefix.  1 <= need <= n.  Every thread of the block must call it.
+template <typename KeyT, typename Fetch>
+__device__ void block_radix_select(Fetch fetch, int n, int need, KeyT &prefix_out, KeyT &mask_out,
+                                   unsigned *hist, unsigned *misc) {
+  constexpr int BITS = sizeof(KeyT) * 8;
+  KeyT prefix = 0, mask = 0;
+  unsigned remaining = static_cast<unsigned>(need);
+  for (int shift = BITS - 8; shift >= 0; shift -= 8) {
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const KeyT k = fetch(i);
+      if ((k & mask) == prefix) atomicAdd(&hist[static_cast<unsigned>(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      unsigned local = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) local += hist[255 - 8 * lane - j];
+      unsigned incl = local;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const unsigned excl = incl - local;
+      if (excl < remaining && remaining <= incl) {
+        unsigned c = excl;
+        for (int j = 0; j < 8; ++j) {
+          const int bin = 255 - 8 * lane - j;
+          if (c + hist[bin] >= remaining) {
+            misc[0] = static_cast<unsigned>(bin);
+            misc[1] = remaining - c;
+            misc[2] = hist[bin];
+            break;
+          }
+          c += hist[bin];
+        }
+      }
+    }
+    __syncthreads();
+    const unsigned chosen = misc[0];
+    remaining = misc[1];
+    const unsigned cnt = misc[2];
+    prefix |= static_cast<KeyT>(chosen) << shift;
+    mask |= static_cast<KeyT>(0xFF) << shift;
+    __syncthreads();
+    if (cnt == remaining) break;
+  }
+  prefix_out = prefix;
+  mask_out = mask;
+}
+
+// ------------------------------------------------------------------ threshold
+__global__ void __launch_bounds__(256) threshold_kernel(SelectArgs a) {
+  __shared__ unsigned hist[256];
+  __shared__ unsigned misc[4];
+  const int tl = blockIdx.x;
+  if (threadIdx.x == 0) {
+    a.cand_count[tl] = 0;
+    if (tl == 0) {
+      a.fb_counters[0] = 0;
+      a.fb_counters[1] = 0;
+    }
+  }
+  const int nvis = a.q_pos0 + tl + 1;
+  const int need = min(a.topk, nvis);
+  unsigned tau = 0u;  // key 0: every score passes
+  if (a.dense != nullptr && nvis > a.cap && a.n_samples > 0) {
+    const double z = 5.0;
+    const double x = static_cast<double>(need) * a.n_samples / nvis;
+    const double rt = z / 2.0 + sqrt(z * z / 4.0 + x);
+    const double rd = ceil(rt * rt);
+    if (rd < a.n_samples) {
+      const int r = static_cast<int>(rd);
+      const float *row = a.dense + static_cast<long long>(tl) * a.dense_ld;
+      unsigned prefix, mask;
+      block_radix_select<unsigned>([&](int i) { return float_order_key(row[i]); }, a.n_samples, r, prefix, mask,
+                                   hist, misc);
+      tau = prefix;
+    }
+  }
+  if (threadIdx.x == 0) a.tau[tl] = tau;
+}
+
+// Bitonic sort of n (power of two) 64-bit values in shared memory, ascending.
+__device__ void block_bitonic_sort(unsigned long long *v, int n) {
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int p = i ^ j;
+        if (p > i) {
+          const bool up = (i & k) == 0;
+          const unsigned long long x = v[i], y = v[p];
+          if ((x > y) == up) {
+            v[i] = y;
+            v[p] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// ------------------------------------------------------------------ select
+__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
+  __shared__ unsigned hist[256];
+  __shared__ unsigned misc[4];
+  __shared__ unsigned long long sortbuf[kMaxTopk];  // (key index << 32) | score key
+  __shared__ int nsel;
+  const int tl = blockIdx.x;
+  const int t = a.t0 + tl;
+  const int nvis = a.q_pos0 + tl + 1;
+  const int need = min(a.topk, nvis);
+  const int count = a.cand_count[tl];
+  if (count > a.cap || count < need) {
+    if (threadIdx.x == 0) {
+      const int pos = atomicAdd(&a.fb_counters[0], 1);
+      a.fb_list[pos] = tl;
+    }
+    return;
+  }
+  const unsigned long long *cand = a.cand + static_cast<long long>(tl) * a.cap;
+  unsigned long long prefix = 0, mask = 0;
+  if (count > need) {
+    block_radix_select<unsigned long long>([&](int i) { return cand[i]; }, count, need, prefix, mask, hist, misc);
+  }
+  if (threadIdx.x == 0) nsel = 0;
+  int npow = 1;
+  while (npow < need) npow <<= 1;
+  for (int i = threadIdx.x; i < npow; i += blockDim.x) sortbuf[i] = ~0ull;
+  __syncthreads();
+  for (int i = threadIdx.x; i < count; i += blockDim.x) {
+    const unsigned long long k = cand[i];
+    if (k >= prefix) {
+      const int p = atomicAdd(&nsel, 1);
+      const unsigned idx = ~static_cast<unsigned>(k & 0xFFFFFFFFull);
+      if (p < npow) sortbuf[p] = (static_cast<unsigned long long>(idx) << 32) | (k >> 32);
+    }
+  }
+  __syncthreads();
+  if (nsel != need) {
+    if (threadIdx.x == 0) atomicOr(a.status, DEV_OVERFLOW);
+  }
+  block_bitonic_sort(sortbuf, npow);
+  int32_t *out = a.topk_idx + static_cast<long long>(t) * a.topk;
+  float *osc = a.topk_score ? a.topk_score + static_cast<long long>(t) * a.topk : nullptr;
+  for (int j = threadIdx.x; j < a.topk; j += blockDim.x) {
+    if (j < need) {
+      const unsigned long long v = sortbuf[j];
+      out[j] = static_cast<int32_t>(v >> 32);
+      if (osc) osc[j] = order_key_float(static_cast<unsigned>(v & 0xFFFFFFFFull));
+    } else {
+      out[j] = -1;
+      if (osc) osc[j] = -INFINITY;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ fallback
+__device__ __forceinline__ float idx_elem(const void *base, long long i, int fp8) {
+  if (fp8) {
+    const __nv_fp8_storage_t b = static_cast<const unsigned char *>(base)[i];
+    return __half2float(__half(__nv_cvt_fp8_to_halfraw(b, __NV_E4M3)));
+  }
+  const unsigned short b = static_cast<const unsigned short *>(base)[i];
+  return __uint_as_float(static_cast<unsigned>(b) << 16);
+}
+
+__global__ void __launch_bounds__(kSelThreads) fallback_kernel(SelectArgs a) {
+  extern __shared__ float fb_smem[];
+  __shared__ unsigned hist[256];
+  __shared__ unsigned misc[4];
+  __shared__ int job;
+  __shared__ int warp_cnt[kSelThreads / 32];
+  __shared__ int warp_off[kSelThreads / 32];
+  __shared__ int base_s;
+  float *q_s = fb_smem;                       // [H_I][D_I]
+  float *w_s = fb_smem + a.H_I * a.D_I;        // [H_I]
+  float *scores = a.fb_scratch + static_cast<long long>(blockIdx.x) * a.N;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  while (true) {
+    __syncthreads();
+    if (threadIdx.x == 0) job = atomicAdd(&a.fb_counters[1], 1);
+    __syncthreads();
+    if (job >= *reinterpret_cast<volatile int *>(&a.fb_counters[0])) break;
+    const int tl = a.fb_list[job];
+    const int t = a.t0 + tl;
+    const int nvis = a.q_pos0 + tl + 1;
+    const int need = min(a.topk, nvis);
+    for (int i = threadIdx.x; i < a.H_I * a.D_I; i += blockDim.x)
+      q_s[i] = idx_elem(a.q_idx, static_cast<long long>(t) * a.H_I * a.D_I + i, a.fp8);
+    for (int i = threadIdx.x; i < a.H_I; i += blockDim.x) w_s[i] = a.w[static_cast<long long>(t) * a.H_I + i];
+    __syncthreads();
+    for (int s = threadIdx.x; s < nvis; s += blockDim.x) {
+      float kr[128];
+      for (int d = 0; d < a.D_I; ++d) kr[d] = idx_elem(a.k_idx, static_cast<long long>(s) * a.D_I + d, a.fp8);
+      float score = 0.0f;
+      for (int h = 0; h < a.H_I; ++h) {
+        float dot = 0.0f;
+        for (int d = 0; d < a.D_I; ++d) dot = fmaf(q_s[h * a.D_I + d], kr[d], dot);
+        score = fmaf(w_s[h], fmaxf(dot, 0.0f), score);
+      }
+      scores[s] = score;
+    }
+    __syncthreads();
+    auto key_of = [&](int s) {
+      return (static_cast<unsigned long long>(float_order_key(scores[s])) << 32) |
+             static_cast<unsigned>(~static_cast<unsigned>(s));
+    };
+    unsigned long long prefix = 0, mask = 0;
+    if (nvis > need) block_radix_select<unsigned long long>(key_of, nvis, need, prefix, mask, hist, misc);
+    if (threadIdx.x == 0) base_s = 0;
+    __syncthreads();
+    int32_t *out = a.topk_idx + static_cast<long long>(t) * a.topk;
+    float *osc = a.topk_score ? a.topk_score + static_cast<long long>(t) * a.topk : nullptr;
+    for (int s0 = 0; s0 < nvis; s0 += blockDim.x) {
+      const int s = s0 + threadIdx.x;
+      const bool sel = (s < nvis) && (key_of(min(s, nvis - 1)) >= prefix);
+      const unsigned bal = __ballot_sync(0xffffffffu, sel);
+      if (lane == 0) warp_cnt[warp] = __popc(bal);
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int w = 0; w < kSelThreads / 32; ++w) {
+          warp_off[w] = acc;
+          acc += warp_cnt[w];
+        }
+        misc[3] = static_cast<unsigned>(acc);
+      }
+      __syncthreads();
+      if (sel) {
+        const int pos = base_s + warp_off[warp] + __popc(bal & ((1u << lane) - 1u));
+        if (pos < need) {
+          out[pos] = s;
+          if (osc) osc[pos] = scores[s];
+        }
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) base_s += static_cast<int>(misc[3]);
+      __syncthreads();
+    }
+    if (threadIdx.x == 0 && base_s != need) atomicOr(a.status, DEV_OVERFLOW);
+    for (int j = need + threadIdx.x; j < a.topk; j += blockDim.x) {
+      out[j] = -1;
+      if (osc) osc[j] = -INFINITY;
+    }
+  }
+}
+
+cudaError_t launch_threshold(const SelectArgs &a, cudaStream_t stream) {
+  threshold_kernel<<<a.Lb, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream) {
+  select_kernel<<<a.Lb, kSelThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fallback(const SelectArgs &a, cudaStream_t stream) {
+  const int smem = (a.H_I * a.D_I + a.H_I) * static_cast<int>(sizeof(float));
+  fallback_kernel<<<a.fb_slots, kSelThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

@@ -1,0 +1,173 @@
+/*
+ * dsa.h -- C ABI of libdsa.so: the prefill hot path of DeepSeek Sparse
+ * Attention (DSA) on NVIDIA B200 (sm_100a).
+ *
+ * The path has three stages per query token t of a prefill chunk:
+ *
+ *   1. Lightning-indexer scores over every causally visible cached key s,
+ *        I[t,s] = sum_h w[t,h] * ReLU(q_idx[t,h,:] . k_idx[s,:]),
+ *      ReLU per indexer head before the signed head weight; one indexer key
+ *      per position shared by all indexer heads.
+ *      (mlx-lm PR #1997, "GLM prefill now attends only to the keys its indexer
+ *      picks", section "How it works": the indexer scores each query against
+ *      every key with 32 heads and keeps the top-k keys per query.)
+ *   2. Exact top-k selection per query without an L x N score tensor in
+ *      memory: a pruned candidate write-back that still returns the exact
+ *      top-k (LiteTopK, arXiv 2607.11976, Abstract).  Ties go to the smaller
+ *      key index.  The result is an int32 [L, topk] index tensor, each row in
+ *      ascending key order, -1 where a query sees fewer than topk keys
+ *      (llama.cpp PR #25917, discussion: sparse index mask, -1 = masked).
+ *   3. Absorbed-MLA attention over only the gathered keys: each key is the
+ *      576-wide joined cache row (512 latent + 64 rope), one gathered block is
+ *      shared by all heads, the value is the 512-wide latent part
+ *      (mlx-lm PR #1997, "How it works").
+ *
+ * Conventions for every entry point
+ *   - Query t of a chunk sits at position q_pos0 + t and sees keys 0..q_pos0+t
+ *     (inclusive causality, position == key index).  0 <= q_pos0, q_pos0+L <= N.
+ *   - All tensor arguments are DEVICE pointers to contiguous row-major
+ *     buffers owned by the caller; the library allocates no device memory and
+ *     keeps no state between calls.  Pointers must be 16-byte aligned.
+ *   - bf16 / fp8 buffers are passed as raw bits (uint16 / uint8 storage).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Argument errors are returned before anything is
+ *     launched; a failed launch returns DSA_ERR_CUDA.  Device-side conditions
+ *     (a wait that timed out, an out-of-range index) are recorded in the
+ *     workspace's status word and read back with dsa_workspace_status().
+ *   - No function aborts the process or throws across the ABI.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1, /* bad pointer, size or shape */
+  DSA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. H_I, D_I, topk) */
+  DSA_ERR_WORKSPACE = 3,   /* workspace missing or too small */
+  DSA_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
+  DSA_ERR_INTERNAL = 5     /* device status word reports a failure */
+} dsa_status_t;
+
+typedef enum {
+  DSA_BF16 = 0,    /* bfloat16 */
+  DSA_FP8_E4M3 = 1 /* OCP FP8 E4M3FN, unit scale */
+} dsa_dtype_t;
+
+typedef struct CUstream_st *dsa_stream_t; /* same type as cudaStream_t */
+
+/* Version of this ABI (incremented on incompatible change). */
+int dsa_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *dsa_status_string(dsa_status_t status);
+
+/*
+ * Workspace (bytes) that dsa_indexer_topk needs for these sizes.  A larger
+ * buffer is fine.  A smaller one that still holds the fixed part shrinks the
+ * per-query candidate capacity; queries whose candidates do not fit are then
+ * resolved by the exact fallback (slower, same result).  Returns 0 for
+ * invalid sizes.
+ */
+size_t dsa_indexer_topk_workspace(int L, int N, int H_I, int D_I, int topk, dsa_dtype_t dtype);
+
+/*
+ * Stages 1+2: lightning-indexer scores and exact top-k per query.
+ *
+ *   q_idx      [L, H_I, D_I]  indexer queries, dtype bits
+ *   k_idx      [N, D_I]       indexer key cache, dtype bits
+ *   w          [L, H_I]       fp32 head weights (signed)
+ *   topk_idx   [L, topk]      out: int32 selected keys, ascending, -1 padded
+ *   topk_score [L, topk]      out (optional, may be NULL): fp32 indexer score
+ *                             of each selected key, -inf for padding
+ *   workspace                 device scratch, workspace_bytes long
+ *
+ * Supported: D_I = 128 with H_I in {4, 8, 16, 32} (bf16 or fp8), D_I = 64 with
+ * H_I in {4, 32} (bf16); 1 <= topk <= 4096.  Queries are processed in blocks of
+ * up to 1,024 (mlx-lm PR #1997, "How it works": long chunks split into query
+ * blocks); the result does not depend on the blocking.
+ */
+dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype, int L,
+                              int N, int H_I, int D_I, int q_pos0, int topk, int32_t *topk_idx, float *topk_score,
+                              void *workspace, size_t workspace_bytes, dsa_stream_t stream);
+
+/* Workspace (bytes) for dsa_sparse_mla_prefill: the status word only. */
+size_t dsa_sparse_mla_workspace(int L, int H, int topk);
+
+/*
+ * Stage 3: sparse absorbed-MLA attention.
+ *
+ *   q        [L, H, 576]  bf16: per head 512 latent then 64 rope columns
+ *   kv       [N, 576]     bf16 joined cache: 512 latent then 64 rope columns
+ *   topk_idx [L, topk]    int32 keys per query; -1 entries are skipped; any
+ *                         order; values >= N are skipped and flagged
+ *   out      [L, H, 512]  out: bf16 attention output
+ *   lse      [L, H]       out (optional, may be NULL): fp32 natural-log
+ *                         log-sum-exp of the scaled logits, -inf if no key
+ *
+ *   z_j = scale * (q_lat . kv_lat[i_j] + q_rope . k_rope[i_j]);
+ *   out = sum_j softmax(z)_j * kv_lat[i_j]    (fp32 accumulate, bf16 out)
+ *
+ * Supported: any H >= 1 (processed in groups of 64 heads), topk >= 1.
+ */
+dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, const int32_t *topk_idx, int L, int N, int H,
+                                    int topk, float scale, void *out, float *lse, void *workspace,
+                                    size_t workspace_bytes, dsa_stream_t stream);
+
+/* Workspace (bytes) for dsa_prefill_chunk with these sizes (query_block <= 0
+ * selects 1,024). */
+size_t dsa_prefill_chunk_workspace(int L, int N, int H_I, int D_I, int H, int topk, int query_block,
+                                   dsa_dtype_t dtype, int want_topk_out);
+
+/*
+ * All three stages for one prefill chunk, query block by query block
+ * (query_block <= 0 selects 1,024 queries per block).
+ *
+ *   q_idx, k_idx, w, dtype, H_I, D_I : as dsa_indexer_topk
+ *   q, kv, H, scale                  : as dsa_sparse_mla_prefill
+ *   topk_idx_out [L, topk]           : optional (may be NULL) selected keys;
+ *                                      when NULL they live in the workspace
+ *   out [L, H, 512], lse [L, H]      : as dsa_sparse_mla_prefill (lse optional)
+ *
+ * want_topk_out of the workspace query must be 0 when topk_idx_out is NULL.
+ */
+dsa_status_t dsa_prefill_chunk(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
+                               const void *q, const void *kv, int L, int N, int H_I, int D_I, int H, int q_pos0,
+                               int topk, float scale, int query_block, int32_t *topk_idx_out, void *out, float *lse,
+                               void *workspace, size_t workspace_bytes, dsa_stream_t stream);
+
+/*
+ * dsa_prefill_chunk, additionally recording CUDA events on `stream` between
+ * its stages (a profiling aid; the computation is identical).  `events` holds
+ * n_events >= 7 * ceil(L / query_block) cudaEvent_t handles; for query block b,
+ * events[7b + 0..6] are recorded before the pilot pass, after the pilot pass,
+ * after the threshold kernel, after the main indexer pass, after the
+ * selection, after the exact fallback and after the attention kernel.
+ */
+dsa_status_t dsa_prefill_chunk_profiled(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
+                                        const void *q, const void *kv, int L, int N, int H_I, int D_I, int H,
+                                        int q_pos0, int topk, float scale, int query_block, int32_t *topk_idx_out,
+                                        void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                        dsa_stream_t stream, void *const *events, int n_events);
+
+/*
+ * Synchronise `stream`, read the device status word at the start of a
+ * workspace used by the calls above and store it in *flags (bit 0: a wait
+ * timed out, bit 1: an index outside [0, N) reached the attention stage,
+ * bit 2: an internal selection count mismatch).  Returns DSA_OK when the word
+ * is zero, DSA_ERR_INTERNAL when it is not, DSA_ERR_CUDA on a CUDA error.
+ * Every entry point clears the word when it starts.
+ */
+dsa_status_t dsa_workspace_status(const void *workspace, dsa_stream_t stream, unsigned *flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

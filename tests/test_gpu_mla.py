@@ -1,0 +1,112 @@
+"""Parity of the CUDA sparse absorbed-MLA attention (dsa_sparse_mla_prefill) with the CPU oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import deepseek_sparse_attention_relu_b200 as dsa
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 1e-2
+MAX_ABS = 3e-2
+
+
+def make(N, L, H, seed, lat_std=0.5, rope_std=0.5):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(L, H, 576, generator=g)
+    q[..., :512] *= lat_std
+    q[..., 512:] *= rope_std
+    kv = torch.randn(N, 576, generator=g)
+    kv[:, :512] *= lat_std
+    kv[:, 512:] *= rope_std
+    return q.to(torch.bfloat16).contiguous(), kv.to(torch.bfloat16).contiguous()
+
+
+def random_selection(N, L, topk, seed, pad=0, q_pos0=None):
+    rng = np.random.default_rng(seed)
+    q_pos0 = N - L if q_pos0 is None else q_pos0
+    idx = np.full((L, topk), -1, dtype=np.int32)
+    for t in range(L):
+        nvis = q_pos0 + t + 1
+        k = min(topk - pad, nvis)
+        idx[t, :k] = np.sort(rng.choice(nvis, k, replace=False))
+    return idx
+
+
+def run_mla(q, kv, idx, scale):
+    dev = torch.device("cuda")
+    L, H, _ = q.shape
+    out = torch.full((L, H, 512), float("nan"), dtype=torch.bfloat16, device=dev)
+    lse = torch.full((L, H), float("nan"), dtype=torch.float32, device=dev)
+    ws = dsa.alloc_workspace(dsa.dsa_sparse_mla_workspace(L, H, idx.shape[1]), dev)
+    dsa.dsa_sparse_mla_prefill(q.to(dev), kv.to(dev), torch.from_numpy(idx).to(dev), scale, out, lse, workspace=ws)
+    assert dsa.dsa_workspace_status(ws) == 0
+    return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def check(q, kv, idx, scale, rows=None):
+    out, lse = run_mla(q, kv, idx, scale)
+    L, H, _ = q.shape
+    pb = oracle.Problem(None, None, None, 0, L, kv.shape[0], 1, 1, 0, idx.shape[1], q=q.view(torch.uint16),
+                        kv=kv.view(torch.uint16), H=H, scale=scale)
+    rows = range(L) if rows is None else rows
+    res = oracle.map_rows(lambda t: (t, *oracle.sparse_mla(pb, t, idx[t])), rows)
+    for t, ro, rl in res:
+        err = np.linalg.norm(out[t] - ro) / max(np.linalg.norm(ro), 1e-30)
+        assert err <= REL_L2, f"query {t}: rel-L2 {err}"
+        assert np.max(np.abs(out[t] - ro)) <= MAX_ABS, f"query {t}: max-abs {np.max(np.abs(out[t] - ro))}"
+        np.testing.assert_allclose(lse[t], rl, rtol=1e-4, atol=1e-3)
+    return out, lse
+
+
+@pytest.mark.parametrize("H", [64, 8, 128, 100])
+def test_heads(H):
+    N, L, topk = 3000, 12, 256
+    q, kv = make(N, L, H, seed=H)
+    idx = random_selection(N, L, topk, seed=H)
+    check(q, kv, idx, 1 / math.sqrt(192))
+
+
+def test_ragged_topk_and_padding():
+    N, L, topk = 5000, 10, 100  # not a multiple of the 64-key tile
+    q, kv = make(N, L, 64, seed=3)
+    idx = random_selection(N, L, topk, seed=3, pad=37)
+    check(q, kv, idx, 1 / math.sqrt(192))
+
+
+def test_unsorted_indices_and_large_scale():
+    N, L, topk = 4096, 6, 512
+    q, kv = make(N, L, 64, seed=5, lat_std=1.0, rope_std=1.0)
+    idx = random_selection(N, L, topk, seed=5)
+    rng = np.random.default_rng(1)
+    for t in range(L):
+        rng.shuffle(idx[t])
+    check(q, kv, idx, 0.25)  # large logits: exercises the running-max rescale
+
+
+def test_single_key_is_exact_and_no_key_is_zero():
+    N, L, topk = 1000, 3, 64
+    q, kv = make(N, L, 64, seed=9)
+    idx = np.full((L, topk), -1, dtype=np.int32)
+    idx[0, 17] = 123
+    idx[1, 0] = 999
+    out, lse = run_mla(q, kv, idx, 1 / math.sqrt(192))
+    assert np.array_equal(out[0], np.broadcast_to(kv[123, :512].float().numpy(), (64, 512)))
+    assert np.array_equal(out[1], np.broadcast_to(kv[999, :512].float().numpy(), (64, 512)))
+    assert np.all(out[2] == 0.0) and np.all(np.isneginf(lse[2]))
+
+
+def test_full_selection_matches_dense_causal():
+    """top-k covering every visible key: the sparse path equals dense causal attention (mlx-lm PR #1997 tests)."""
+    N = L = 300
+    q, kv = make(N, L, 64, seed=11)
+    idx = random_selection(N, L, 320, seed=0, q_pos0=0)  # pads every row
+    out, _ = run_mla(q, kv, idx, 1 / math.sqrt(192))
+    pb = oracle.Problem(None, None, None, 0, L, N, 1, 1, 0, 320, q=q.view(torch.uint16), kv=kv.view(torch.uint16),
+                        H=64, scale=1 / math.sqrt(192))
+    for t in (0, 1, 150, 299):
+        ro, _ = oracle.dense_causal_mla(pb, t)
+        assert np.linalg.norm(out[t] - ro) / np.linalg.norm(ro) <= REL_L2
