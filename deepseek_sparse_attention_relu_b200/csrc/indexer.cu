@@ -42,22 +42,53 @@ struct IdxCfg {
   static constexpr int QG = BN / HI;
   static constexpr int K_TILE = BM * ROW_BYTES;
   static constexpr int Q_TILE = BN * ROW_BYTES;
-  static constexpr int STAGES = (K_TILE <= 16384) ? 8 : 4;
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = 64 + EPI_WARPS * 32;
+  static constexpr int QH = QG / 2;                       // queries per epilogue warp
+  static constexpr int SB = (256 / QH) < 32 ? 32 : (256 / QH);  // staged candidates per (warp, query)
+  static constexpr int STG_BYTES = EPI_WARPS * QH * SB * 8;
+  static constexpr int SMEM_BUDGET = 224 * 1024;
+  static constexpr int FIXED = Q_TILE + STG_BYTES + 2 * EPI_WARPS * 128 * 4 + 2048;
+  static constexpr int STAGES_FIT = (SMEM_BUDGET - FIXED) / K_TILE;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   // shared memory carve-up (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_TILE;
-  static constexpr int OFF_W = OFF_K + STAGES * K_TILE;       // [EPI_WARPS][128] floats
-  static constexpr int OFF_TAU = OFF_W + EPI_WARPS * 128 * 4;  // [EPI_WARPS][QG/2] floats
+  static constexpr int OFF_STG = OFF_K + STAGES * K_TILE;        // [EPI_WARPS][QH][SB] candidate keys
+  static constexpr int OFF_W = OFF_STG + STG_BYTES;              // [EPI_WARPS][128] floats
+  static constexpr int OFF_TAU = OFF_W + EPI_WARPS * 128 * 4;    // [EPI_WARPS][QH] float thresholds
   static constexpr int OFF_BAR = OFF_TAU + EPI_WARPS * 128 * 4;  // mbarriers
   static constexpr int NBAR = 2 * STAGES + 2 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // tmem addr, abort flag, counters
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
+  static_assert(STAGES >= 3, "not enough shared memory for the key pipeline");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(ROW_BYTES % 128 == 0, "indexer rows must be whole 128-byte atoms");
+  static_assert(HI % 4 == 0, "head weights are read four at a time");
   static_assert(QG * HI == BN, "H_I must divide 256");
   static_assert((QG / 2) * HI == 128, "each epilogue half covers 128 columns");
 };
+
+union F2U {
+  float2 f;
+  unsigned long long u;
+};
+
+// Two independent fp32 FMAs in one instruction: {a.x*b.x + c.x, a.y*b.y + c.y}, round to nearest.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  F2U x, y, z, r;
+  x.f = a;
+  y.f = b;
+  z.f = c;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.u) : "l"(x.u), "l"(y.u), "l"(z.u));
+  return r.f;
+}
+
+// Threshold key -> float: a score s passes iff s >= threshold_float(key).  Key 0
+// (and anything at or below the key of -inf) passes every finite score.
+__device__ __forceinline__ float threshold_float(unsigned key) {
+  return key < 0x00800000u ? -INFINITY : order_key_float(key);
+}
 
 // Per-group number of 128-key tiles.
 __device__ __forceinline__ int idx_group_tiles(const IndexerArgs &a, int g, int QG) {
@@ -265,17 +296,44 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     const int ew = warp - 2;          // 0..7
     const int quarter = warp & 3;     // TMEM lane quarter this warp may access
     const int half = ew >> 2;         // which 128 accumulator columns
-    constexpr int QH = C::QG / 2;     // queries per half
+    constexpr int QH = C::QH;         // queries per warp
+    constexpr int SB = C::SB;
     TileCursor c = idx_cursor_begin(a, C::QG);
     int acc = 0, prev_g = -1;
     unsigned acc_phase = 0;
     bool ok = true;
     const unsigned lane_mask_lt = (1u << lane) - 1u;
     float *w_w = w_s + ew * 128;   // this warp's head weights: [QH queries][HI]
-    unsigned *tau_w = reinterpret_cast<unsigned *>(tau_s) + ew * 128;
+    float *tau_w = tau_s + ew * 128;
+    unsigned long long *stg = reinterpret_cast<unsigned long long *>(smem + C::OFF_STG) + ew * QH * SB;
+    int cnt[QH];                   // staged candidates per query (warp-uniform)
+#pragma unroll
+    for (int qq = 0; qq < QH; ++qq) cnt[qq] = 0;
+
+    // Move a query's staged candidates to its global list: one atomic per batch.
+    auto flush = [&](int qq, int gq) {
+      const int n = cnt[qq];
+      if (n == 0) return;
+      const int tl = gq * C::QG + half * QH + qq;
+      __syncwarp();
+      int base = 0;
+      if (lane == 0) base = atomicAdd(&a.cand_count[tl], n);
+      base = __shfl_sync(0xffffffffu, base, 0);
+      for (int i = lane; i < n; i += 32) {
+        const int pos = base + i;
+        if (pos < a.cap) a.cand[static_cast<long long>(tl) * a.cap + pos] = stg[qq * SB + i];
+      }
+      __syncwarp();
+      cnt[qq] = 0;
+    };
+
     while (c.left > 0) {
       const int g = c.g;
       if (g != prev_g) {
+        if (!PILOT && prev_g >= 0) {
+#pragma unroll
+          for (int qq = 0; qq < QH; ++qq) flush(qq, prev_g);
+        }
         // Each warp stages the head weights / thresholds of its own queries
         // (no cross-warp barrier, so an aborting warp cannot strand the others).
         __syncwarp();
@@ -286,7 +344,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
         if (!PILOT) {
           for (int j = lane; j < QH; j += 32) {
             const int tl = g * C::QG + half * QH + j;
-            tau_w[j] = (tl < a.Lb) ? a.tau[tl] : 0xFFFFFFFFu;
+            tau_w[j] = (tl < a.Lb) ? threshold_float(a.tau[tl]) : INFINITY;
           }
         }
         __syncwarp();
@@ -306,38 +364,44 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
       const int key = c.tile * C::BM + quarter * 32 + lane;
 #pragma unroll
       for (int qq = 0; qq < QH; ++qq) {
-        const int qg = half * QH + qq;  // query within the group
-        const int tl = g * C::QG + qg;  // query within the block
-        float score = 0.0f;
+        const int tl = g * C::QG + half * QH + qq;  // query within the block
+        const float4 *wq = reinterpret_cast<const float4 *>(w_w + qq * HI);
+        float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int h = 0; h < HI; ++h) {
-          const int col = qq * HI + h;
-          const float s = __uint_as_float(v[col / 32][col % 32]);
-          score = fmaf(w_w[qq * HI + h], fmaxf(s, 0.0f), score);
+        for (int h4 = 0; h4 < HI / 4; ++h4) {
+          const float4 w4 = wq[h4];
+          const int col = qq * HI + 4 * h4;
+          const float r0 = fmaxf(__uint_as_float(v[(col + 0) / 32][(col + 0) % 32]), 0.0f);
+          const float r1 = fmaxf(__uint_as_float(v[(col + 1) / 32][(col + 1) % 32]), 0.0f);
+          const float r2 = fmaxf(__uint_as_float(v[(col + 2) / 32][(col + 2) % 32]), 0.0f);
+          const float r3 = fmaxf(__uint_as_float(v[(col + 3) / 32][(col + 3) % 32]), 0.0f);
+          acc0 = ffma2(make_float2(w4.x, w4.y), make_float2(r0, r1), acc0);
+          acc1 = ffma2(make_float2(w4.z, w4.w), make_float2(r2, r3), acc1);
         }
+        const float score = (acc0.x + acc1.x) + (acc0.y + acc1.y);
         if (PILOT) {
           if (tl < a.Lb && key < a.n_keys) a.dense[static_cast<long long>(tl) * a.dense_ld + key] = score;
         } else {
-          const bool pass = (tl < a.Lb) && (key <= a.q_pos0 + tl) && (float_order_key(score) >= tau_w[qq]);
+          const bool pass = (tl < a.Lb) && (key <= a.q_pos0 + tl) && (score >= tau_w[qq]);
           const unsigned m = __ballot_sync(0xffffffffu, pass);
           if (m) {
-            const int leader = __ffs(m) - 1;
-            int base = 0;
-            if (lane == leader) base = atomicAdd(&a.cand_count[tl], __popc(m));
-            base = __shfl_sync(0xffffffffu, base, leader);
+            const int n = __popc(m);
+            if (cnt[qq] + n > SB) flush(qq, g);
             if (pass) {
-              const int pos = base + __popc(m & lane_mask_lt);
-              if (pos < a.cap) {
-                const unsigned long long k64 = (static_cast<unsigned long long>(float_order_key(score)) << 32) |
-                                               static_cast<unsigned>(~static_cast<unsigned>(key));
-                a.cand[static_cast<long long>(tl) * a.cap + pos] = k64;
-              }
+              const unsigned long long k64 = (static_cast<unsigned long long>(float_order_key(score)) << 32) |
+                                             static_cast<unsigned>(~static_cast<unsigned>(key));
+              stg[qq * SB + cnt[qq] + __popc(m & lane_mask_lt)] = k64;
             }
+            cnt[qq] += n;
           }
         }
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       idx_cursor_next(c, a, C::QG);
+    }
+    if (ok && !PILOT && prev_g >= 0) {
+#pragma unroll
+      for (int qq = 0; qq < QH; ++qq) flush(qq, prev_g);
     }
     if (!ok) {
       if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
@@ -375,20 +439,18 @@ cudaError_t launch_indexer(const CUtensorMap &tq, const CUtensorMap &tk, const I
   DSA_IDX_CASE(128, 32, false)
   DSA_IDX_CASE(128, 32, true)
   DSA_IDX_CASE(64, 4, false)
-  DSA_IDX_CASE(128, 4, false)
   DSA_IDX_CASE(64, 32, false)
   DSA_IDX_CASE(128, 16, false)
   DSA_IDX_CASE(128, 16, true)
   DSA_IDX_CASE(128, 8, false)
   DSA_IDX_CASE(128, 8, true)
-  DSA_IDX_CASE(128, 4, true)
 #undef DSA_IDX_CASE
   return cudaErrorInvalidValue;
 }
 
 bool indexer_supported(int D_I, int H_I, bool fp8) {
-  if (fp8) return D_I == 128 && (H_I == 32 || H_I == 16 || H_I == 8 || H_I == 4);
-  if (D_I == 128) return H_I == 32 || H_I == 16 || H_I == 8 || H_I == 4;
+  if (fp8) return D_I == 128 && (H_I == 32 || H_I == 16 || H_I == 8);
+  if (D_I == 128) return H_I == 32 || H_I == 16 || H_I == 8;
   if (D_I == 64) return H_I == 32 || H_I == 4;
   return false;
 }

@@ -128,16 +128,38 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int at = 0; at < ATOMS; ++at) tma_load_2d(q_s + at * ATOM_BYTES, &tmap_q, q_full, at * 64, row0);
     }
     const int32_t *idx_row = a.topk_idx + static_cast<long long>(t) * a.topk;
+    const bool vec_idx = (a.topk % 4) == 0;
+    // Lanes 0..15 own keys 4l..4l+3 of a tile.  The indices of tile j+1 are
+    // loaded while tile j waits for its stage, so their latency stays hidden.
+    auto load_idx = [&](int j, int (&r)[4]) {
+      r[0] = r[1] = r[2] = r[3] = -1;
+      if (lane < 16 && j < ntiles) {
+        const int pos = j * BK + lane * 4;
+        if (vec_idx && pos + 3 < a.topk) {
+          const int4 v = *reinterpret_cast<const int4 *>(idx_row + pos);
+          r[0] = v.x;
+          r[1] = v.y;
+          r[2] = v.z;
+          r[3] = v.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (pos + e < a.topk) r[e] = idx_row[pos + e];
+        }
+      }
+    };
+    int cur[4], nxt[4];
+    load_idx(0, cur);
     for (int j = 0; j < ntiles; ++j) {
       const int st = j & 1;
+      load_idx(j + 1, nxt);
       if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1u, abort_flag)) { ok = false; break; }
       int r[4];
       unsigned bits = 0;
       if (lane < 16) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int pos = j * BK + lane * 4 + e;
-          const int v = pos < a.topk ? idx_row[pos] : -1;
+          const int v = cur[e];
           const bool good = v >= 0 && v < a.N;
           if (v >= a.N || v < -1) atomicOr(a.status, DEV_BAD_INDEX);
           r[e] = good ? v : 0;
@@ -164,6 +186,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           tma_gather4(dst + at * ATOM_BYTES, &tmap_kv, &kv_full[st], at * 64, r[0], r[1], r[2], r[3]);
       }
       ++issued;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) cur[e] = nxt[e];
     }
     if (!ok) {
       if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
@@ -197,39 +221,54 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_commit(&kv_empty[jj & 1]);
       tc_commit(p_free);
     };
-    for (int j = 0; ok && j < ntiles; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(&kv_full[st], (j >> 1) & 1u, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(&s_free[st], ((j >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-      tc_fence_after();
+    // Event-driven issue: O += P V for tile np as soon as its P is written (it
+    // frees a gather stage), otherwise S = Q K^T for tile nq once its keys have
+    // landed and its S buffer is free.  Lane 0 polls, the warp follows.
+    int nq = 0, np = 0;
+    bool idle = false;
+    unsigned long long t_idle = 0;
+    unsigned spins = 0;
+    while (ok && np < ntiles) {
+      int action = 0;
       if (lane == 0) {
-        const unsigned k_base = smem_u32(kv_s + st * KV_BYTES);
-        for (int at = 0; at < ATOMS; ++at) {
+        if (np < nq && mbar_try_wait(p_full, np & 1u))
+          action = 1;
+        else if (nq < ntiles && mbar_try_wait(&kv_full[nq & 1], (nq >> 1) & 1u) &&
+                 mbar_try_wait(&s_free[nq & 1], ((nq >> 1) & 1u) ^ 1u))
+          action = 2;
+      }
+      action = __shfl_sync(0xffffffffu, action, 0);
+      if (action == 1) {
+        tc_fence_after();
+        if (lane == 0) issue_pv(np);
+        __syncwarp();
+        ++np;
+        idle = false;
+      } else if (action == 2) {
+        tc_fence_after();
+        if (lane == 0) {
+          const int st = nq & 1;
+          const unsigned k_base = smem_u32(kv_s + st * KV_BYTES);
+          for (int at = 0; at < ATOMS; ++at) {
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t qd = smem_desc_sw128(q_base + at * ATOM_BYTES + ks * 32, 16, 1024);
-            const uint64_t kd = smem_desc_sw128(k_base + at * ATOM_BYTES + ks * 32, 16, 1024);
-            mma_bf16_ss(s_col + st * 64, qd, kd, idesc_qk, (at | ks) ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t qd = smem_desc_sw128(q_base + at * ATOM_BYTES + ks * 32, 16, 1024);
+              const uint64_t kd = smem_desc_sw128(k_base + at * ATOM_BYTES + ks * 32, 16, 1024);
+              mma_bf16_ss(s_col + st * 64, qd, kd, idesc_qk, (at | ks) ? 1u : 0u);
+            }
           }
+          tc_commit(&s_full[st]);
+          *reinterpret_cast<volatile int *>(consumed) = nq + 1;
         }
-        tc_commit(&s_full[st]);
-        *reinterpret_cast<volatile int *>(consumed) = j + 1;
-      }
-      __syncwarp();
-      if (j > 0) {
-        if (!mbar_wait(p_full, (j - 1) & 1u, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        if (lane == 0) issue_pv(j - 1);
         __syncwarp();
-      }
-    }
-    if (ok) {
-      if (mbar_wait(p_full, (ntiles - 1) & 1u, abort_flag)) {
-        tc_fence_after();
-        if (lane == 0) issue_pv(ntiles - 1);
-        __syncwarp();
-      } else {
-        ok = false;
+        ++nq;
+        idle = false;
+      } else if (!idle) {
+        idle = true;
+        t_idle = globaltimer();
+        spins = 0;
+      } else if ((++spins & 63u) == 0) {
+        if (*abort_flag || globaltimer() - t_idle > kWaitLimitNs) ok = false;
       }
     }
     if (!ok) {

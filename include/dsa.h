@@ -88,7 +88,7 @@ size_t dsa_indexer_topk_workspace(int L, int N, int H_I, int D_I, int topk, dsa_
  *                             of each selected key, -inf for padding
  *   workspace                 device scratch, workspace_bytes long
  *
- * Supported: D_I = 128 with H_I in {4, 8, 16, 32} (bf16 or fp8), D_I = 64 with
+ * Supported: D_I = 128 with H_I in {8, 16, 32} (bf16 or fp8), D_I = 64 with
  * H_I in {4, 32} (bf16); 1 <= topk <= 4096.  Queries are processed in blocks of
  * up to 1,024 (mlx-lm PR #1997, "How it works": long chunks split into query
  * blocks); the result does not depend on the blocking.
