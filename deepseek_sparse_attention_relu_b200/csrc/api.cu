@@ -9,7 +9,7 @@
 #include <cstdint>
 #include <cstring>
 
-#include "../../include/dsa.h"
+#include "dsa.h"
 #include "dsa_internal.h"
 
 namespace {
@@ -261,16 +261,16 @@ dsa_status_t check_mla_args(const MlaProblem &p) {
   return DSA_OK;
 }
 
-bool make_mla_maps(const MlaProblem &p, CUtensorMap *tq, CUtensorMap *tkv) {
+bool make_mla_maps(const MlaProblem &p, CUtensorMap *tq) {
   return make_map_2d(tq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 576, static_cast<uint64_t>(p.L) * p.H, 576 * 2, 64,
-                     64) &&
-         make_map_2d(tkv, p.kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 576, p.N, 576 * 2, 64, 1);
+                     64);
 }
 
-dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, const CUtensorMap &tkv, unsigned *status,
-                           int t0, int Lq, cudaStream_t stream) {
+dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, unsigned *status, int t0, int Lq,
+                           cudaStream_t stream) {
   MlaArgs a{};
   a.topk_idx = p.topk_idx;
+  a.kv = p.kv;
   a.out = static_cast<uint16_t *>(p.out);
   a.lse = p.lse;
   a.status = status;
@@ -281,7 +281,7 @@ dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, const CUt
   a.t0 = t0;
   a.Lq = Lq;
   a.scale_log2 = p.scale * 1.4426950408889634f;
-  return launch_sparse_mla(tq, tkv, a, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  return launch_sparse_mla(tq, a, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // namespace
@@ -343,11 +343,11 @@ dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, const int32_t
   if (st != DSA_OK) return st;
   if (workspace == nullptr || workspace_bytes < kHeaderBytes) return DSA_ERR_WORKSPACE;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  CUtensorMap tq, tkv;
-  if (!make_mla_maps(p, &tq, &tkv)) return DSA_ERR_CUDA;
+  CUtensorMap tq;
+  if (!make_mla_maps(p, &tq)) return DSA_ERR_CUDA;
   unsigned *status = static_cast<unsigned *>(workspace);
   if (cudaMemsetAsync(status, 0, kHeaderBytes, stream) != cudaSuccess) return DSA_ERR_CUDA;
-  return run_mla_block(p, tq, tkv, status, 0, L, stream);
+  return run_mla_block(p, tq, status, 0, L, stream);
 }
 
 size_t dsa_prefill_chunk_workspace(int L, int N, int H_I, int D_I, int H, int topk, int query_block,
@@ -391,8 +391,8 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, const floa
   IdxWorkspace ws;
   if (!carve_idx_ws(workspace, idx_bytes, QB, N, &ws)) return DSA_ERR_WORKSPACE;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  CUtensorMap tq, tk, mq, mkv;
-  if (!make_indexer_maps(ip, &tq, &tk) || !make_mla_maps(mp, &mq, &mkv)) return DSA_ERR_CUDA;
+  CUtensorMap tq, tk, mq;
+  if (!make_indexer_maps(ip, &tq, &tk) || !make_mla_maps(mp, &mq)) return DSA_ERR_CUDA;
   const int nblocks = (L + QB - 1) / QB;
   if (events != nullptr && n_events < 7 * nblocks) return DSA_ERR_INVALID_ARG;
   if (cudaMemsetAsync(ws.status, 0, kHeaderBytes, stream) != cudaSuccess) return DSA_ERR_CUDA;
@@ -408,7 +408,7 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, const floa
     }
     st = run_indexer_block(bp, tq, tk, ws, t0, Lb, stream, ev);
     if (st != DSA_OK) return st;
-    st = run_mla_block(bm, mq, mkv, ws.status, t0, Lb, stream);
+    st = run_mla_block(bm, mq, ws.status, t0, Lb, stream);
     if (st != DSA_OK) return st;
     if (!mark(ev, 6, stream)) return DSA_ERR_CUDA;
   }

@@ -58,6 +58,7 @@ cudaError_t launch_fallback(const SelectArgs &a, cudaStream_t stream);
 // Sparse absorbed-MLA attention.
 struct MlaArgs {
   const int32_t *topk_idx;        // [L, topk]
+  const void *kv;                 // [N, 576] bf16 joined cache
   uint16_t *out;                  // [L, H, 512] bf16 bits
   float *lse;                     // [L, H] or nullptr
   unsigned *status;
@@ -66,6 +67,6 @@ struct MlaArgs {
   float scale_log2;               // softmax scale * log2(e)
 };
 
-cudaError_t launch_sparse_mla(const CUtensorMap &tq, const CUtensorMap &tkv, const MlaArgs &a, cudaStream_t stream);
+cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, cudaStream_t stream);
 
 }  // namespace dsa

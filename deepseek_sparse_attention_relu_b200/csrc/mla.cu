@@ -10,8 +10,11 @@
 // Index -1 marks a skipped entry (llama.cpp PR #25917, discussion).
 //
 // B200 mapping.  One CTA per (query, group of 64 heads).  Per 64-key tile:
-//   * TMA tile::gather4 loads the 64 selected rows (9 column atoms of 128 B,
-//     128-byte swizzle) straight into the UMMA operand layout;
+//   * two producer warps, one per stage, gather the 64 selected rows with
+//     16-byte cp.async copies (each 8-lane group moves one 128-byte row
+//     segment, coalesced) straight into the 128-byte-swizzled UMMA operand
+//     layout; a tensor-map gather (tile::gather4) was measured to issue too
+//     slowly for 1,152-byte rows;
 //   * S = Q K^T on tcgen05 (M = 64 heads, N = 64 keys, K = 576), fp32 in TMEM;
 //   * softmax warps read S from TMEM, keep a running max (rescaling the output
 //     only when the max grows by more than 2^8) and write P (bf16) to shared
@@ -20,8 +23,9 @@
 //     V read in place from the gathered tile as an MN-major operand.
 // TMEM: the two 64 x 256 fp32 halves of O sit in the two half-subpartitions
 // (lanes 0-15 and 16-31 of each 32-lane quarter) of columns 0-255, the two S
-// buffers in columns 256-383.  Warp roles: warp 0 gather producer, warp 1 MMA
-// issuer / TMEM owner, warps 2-5 softmax and output.
+// buffers in columns 256-383.  Warp roles: warps 0 and 6 gather producers
+// (stage 0 / stage 1), warp 1 MMA issuer / TMEM owner, warps 2-5 softmax and
+// output.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -41,7 +45,7 @@ constexpr int Q_BYTES = ATOMS * ATOM_BYTES;
 constexpr int KV_BYTES = ATOMS * ATOM_BYTES;
 constexpr int P_BYTES = HT * BK * 2;
 constexpr int STAGES = 2;
-constexpr int THREADS = 192;
+constexpr int THREADS = 224;
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + Q_BYTES;
 constexpr int OFF_P = OFF_KV + STAGES * KV_BYTES;
@@ -58,8 +62,7 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_kv,
-                      MlaArgs a) {
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q, MlaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *q_s = smem + OFF_Q;
@@ -77,7 +80,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
   unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + OFF_MISC + 8);  // [2]
-  int *consumed = reinterpret_cast<int *>(smem + OFF_MISC + 24);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -99,17 +101,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(p_free, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
-    *consumed = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&tmap_q);
-    prefetch_tensormap(&tmap_kv);
-  }
+  if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_q);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -118,87 +116,66 @@ __global__ void __launch_bounds__(THREADS, 1)
   const unsigned o_hi = tmem + (16u << 16);            // lanes 16-31 of each quarter, cols 0-255
   const unsigned s_col = tmem + 256;                   // S buffers: cols 256-319, 320-383
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ gather producer
+  if (warp == 0 || warp == 6) {
+    // ------------------------------------------------------------ gather producers
+    // Producer p owns stage p and fills tiles p, p + 2, p + 4, ...  Lane l moves
+    // the 16-byte column chunk (l % 8) of rows 4g + l / 8 (g = 0..15) for all
+    // 9 column atoms: every 8-lane group reads one whole 128-byte segment.
+    const int p = warp == 0 ? 0 : 1;
+    const int r = lane >> 3, c8 = lane & 7;
     bool ok = true;
-    int issued = 0;
-    if (lane == 0) {
+    if (p == 0 && lane == 0) {
       mbar_arrive_expect_tx(q_full, Q_BYTES);
       const int row0 = t * a.H + hg * HT;
       for (int at = 0; at < ATOMS; ++at) tma_load_2d(q_s + at * ATOM_BYTES, &tmap_q, q_full, at * 64, row0);
     }
     const int32_t *idx_row = a.topk_idx + static_cast<long long>(t) * a.topk;
-    const bool vec_idx = (a.topk % 4) == 0;
-    // Lanes 0..15 own keys 4l..4l+3 of a tile.  The indices of tile j+1 are
-    // loaded while tile j waits for its stage, so their latency stays hidden.
-    auto load_idx = [&](int j, int (&r)[4]) {
-      r[0] = r[1] = r[2] = r[3] = -1;
-      if (lane < 16 && j < ntiles) {
-        const int pos = j * BK + lane * 4;
-        if (vec_idx && pos + 3 < a.topk) {
-          const int4 v = *reinterpret_cast<const int4 *>(idx_row + pos);
-          r[0] = v.x;
-          r[1] = v.y;
-          r[2] = v.z;
-          r[3] = v.w;
-        } else {
+    auto load_idx = [&](int j, int (&v)[16]) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (pos + e < a.topk) r[e] = idx_row[pos + e];
-        }
+      for (int g = 0; g < 16; ++g) {
+        const int pos = j * BK + 4 * g + r;
+        v[g] = (j < ntiles && pos < a.topk) ? idx_row[pos] : -1;
       }
     };
-    int cur[4], nxt[4];
-    load_idx(0, cur);
-    for (int j = 0; j < ntiles; ++j) {
-      const int st = j & 1;
-      load_idx(j + 1, nxt);
-      if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1u, abort_flag)) { ok = false; break; }
-      int r[4];
-      unsigned bits = 0;
-      if (lane < 16) {
+    const uint8_t *kv = static_cast<const uint8_t *>(a.kv);
+    const unsigned stage_base = smem_u32(kv_s + p * KV_BYTES);
+    int cur[16], nxt[16];
+    load_idx(p, cur);
+    for (int j = p; j < ntiles; j += 2) {
+      load_idx(j + 2, nxt);
+      if (!mbar_wait(&kv_empty[p], ((j >> 1) & 1) ^ 1u, abort_flag)) { ok = false; break; }
+      unsigned long long vbits = 0;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int v = cur[e];
-          const bool good = v >= 0 && v < a.N;
-          if (v >= a.N || v < -1) atomicOr(a.status, DEV_BAD_INDEX);
-          r[e] = good ? v : 0;
-          bits |= (good ? 1u : 0u) << e;
-        }
-      }
-      // 64-bit validity mask of this tile: lane l contributes bits 4l..4l+3.
-      unsigned lo = (lane < 8) ? (bits << (4 * lane)) : 0u;
-      unsigned hi = (lane >= 8 && lane < 16) ? (bits << (4 * (lane - 8))) : 0u;
+      for (int g = 0; g < 16; ++g) {
+        const int v = cur[g];
+        const bool good = v >= 0 && v < a.N;
+        if (c8 == 0 && (v >= a.N || v < -1)) atomicOr(a.status, DEV_BAD_INDEX);
+        vbits |= static_cast<unsigned long long>(good ? 1u : 0u) << (4 * g + r);
+        const int row = good ? v : 0;
+        const int key = 4 * g + r;
+        const uint8_t *src = kv + static_cast<long long>(row) * (DIM * 2) + c8 * 16;
+        const unsigned dst = stage_base + key * 128 + ((c8 ^ (key & 7)) << 4);
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        lo |= __shfl_xor_sync(0xffffffffu, lo, off);
-        hi |= __shfl_xor_sync(0xffffffffu, hi, off);
+        for (int at = 0; at < ATOMS; ++at) cp_async_16(dst + at * ATOM_BYTES, src + at * 128);
       }
-      if (lane == 0) {
-        valid_s[st] = (static_cast<unsigned long long>(hi) << 32) | lo;
-        mbar_arrive_expect_tx(&kv_full[st], KV_BYTES);
-      }
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      vbits |= __shfl_xor_sync(0xffffffffu, vbits, 8);
+      vbits |= __shfl_xor_sync(0xffffffffu, vbits, 16);
       __syncwarp();
-      if (lane < 16) {
-        uint8_t *dst = kv_s + st * KV_BYTES + lane * 4 * 128;
-#pragma unroll
-        for (int at = 0; at < ATOMS; ++at)
-          tma_gather4(dst + at * ATOM_BYTES, &tmap_kv, &kv_full[st], at * 64, r[0], r[1], r[2], r[3]);
+      if (lane == 0) {
+        valid_s[p] = vbits;
+        mbar_arrive(&kv_full[p]);
       }
-      ++issued;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) cur[e] = nxt[e];
+      for (int g = 0; g < 16; ++g) cur[g] = nxt[g];
     }
+    cp_async_wait_all();  // never leave with copies in flight
     if (!ok) {
       if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
       *abort_flag = 1;
     }
-    if (lane == 0) {
-      // Never leave with copies in flight.
-      mbar_wait(q_full, 0u, nullptr);
-      const int done = *reinterpret_cast<volatile int *>(consumed);
-      for (int i = done; i < issued; ++i) mbar_wait(&kv_full[i & 1], (i >> 1) & 1u, nullptr);
-    }
+    if (p == 0 && lane == 0) mbar_wait(q_full, 0u, nullptr);
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -258,7 +235,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
           tc_commit(&s_full[st]);
-          *reinterpret_cast<volatile int *>(consumed) = nq + 1;
         }
         __syncwarp();
         ++nq;
@@ -414,12 +390,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace mla
 
-cudaError_t launch_sparse_mla(const CUtensorMap &tq, const CUtensorMap &tkv, const MlaArgs &a, cudaStream_t stream) {
+cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(mla::sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        mla::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(a.Lq, (a.H + mla::HT - 1) / mla::HT);
-  mla::sparse_mla_kernel<<<grid, mla::THREADS, mla::SMEM_BYTES, stream>>>(tq, tkv, a);
+  mla::sparse_mla_kernel<<<grid, mla::THREADS, mla::SMEM_BYTES, stream>>>(tq, a);
   return cudaGetLastError();
 }
 

@@ -1,5 +1,5 @@
 // ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers with bounded
-// waits, TMA tile / gather4 loads, and the tcgen05 tensor-core + tensor-memory
+// waits, TMA tile loads, cp.async copies, and the tcgen05 tensor-core + tensor-memory
 // instructions.  Every wait gives up after a wall-clock limit so that a lost
 // arrival turns into an error status instead of a hung GPU.
 #pragma once
@@ -90,16 +90,12 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
       : "memory");
 }
 
-// Four rows (r0..r3) of a 2D tensor, columns [x, x + box width), into four
-// consecutive box rows at dst.  The tensor map's box must be one row high.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int r0, int r1,
-                                            int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
-      "%4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
+// 16-byte global -> shared copy through L2 (no L1 allocation), asynchronous.
+__device__ __forceinline__ void cp_async_16(unsigned dst_smem, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
 }
+// Wait until every cp.async issued by this thread has landed in shared memory.
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
