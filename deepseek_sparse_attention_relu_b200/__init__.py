@@ -24,7 +24,7 @@ DSA_FP8_E4M3 = 1
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_WORKSPACE",
                 4: "DSA_ERR_CUDA", 5: "DSA_ERR_INTERNAL"}
 
-EXPORTED = ("dsa_version", "dsa_status_string", "dsa_indexer_topk_workspace", "dsa_indexer_topk",
+EXPORTED = ("dsa_version", "dsa_status_string", "dsa_last_error_string", "dsa_indexer_topk_workspace", "dsa_indexer_topk",
             "dsa_sparse_mla_workspace", "dsa_sparse_mla_prefill", "dsa_prefill_chunk_workspace",
             "dsa_prefill_chunk", "dsa_prefill_chunk_profiled", "dsa_workspace_status")
 
@@ -34,7 +34,10 @@ _lib = None
 class DSAError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {lib().dsa_status_string(status).decode()}")
+        msg = lib().dsa_status_string(status).decode()
+        if status == 4:
+            msg += f" ({lib().dsa_last_error_string().decode()})"
+        super().__init__(f"{where}: {msg}")
 
 
 def lib() -> ctypes.CDLL:
@@ -50,6 +53,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_version.argtypes = []
         L.dsa_status_string.restype = ctypes.c_char_p
         L.dsa_status_string.argtypes = [I]
+        L.dsa_last_error_string.restype = ctypes.c_char_p
+        L.dsa_last_error_string.argtypes = []
         L.dsa_indexer_topk_workspace.restype = Z
         L.dsa_indexer_topk_workspace.argtypes = [I, I, I, I, I, I]
         L.dsa_indexer_topk.restype = I

@@ -23,6 +23,16 @@ constexpr int kMinCap = 8192;             // default candidate capacity per quer
 constexpr int kMaxTopk = 4096;
 constexpr size_t kHeaderBytes = 256;      // status word, fallback counters
 
+// The CUDA error behind the calling thread's last DSA_ERR_CUDA (cudaSuccess if none).
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+// True on success; otherwise remembers the error for dsa_last_error_string().
+bool cuda_ok(cudaError_t e) {
+  if (e == cudaSuccess) return true;
+  t_last_cuda_error = e;
+  return false;
+}
+
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -135,7 +145,7 @@ dsa_status_t check_indexer_args(const IndexerProblem &p) {
 // Stages 1+2 for queries [t0, t0 + Lb) of the chunk.
 // Record ev[i] on the stream when profiling events were supplied.
 bool mark(cudaEvent_t *ev, int i, cudaStream_t stream) {
-  return ev == nullptr || ev[i] == nullptr || cudaEventRecord(ev[i], stream) == cudaSuccess;
+  return ev == nullptr || ev[i] == nullptr || cuda_ok(cudaEventRecord(ev[i], stream));
 }
 
 // ev (optional): 6 events recorded before the pilot, after the pilot, after the
@@ -176,8 +186,7 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
     pa.dense_ld = n_samples;
     pa.n_keys = n_samples;
     pa.total_tiles = G * ((n_samples + 127) / 128);
-    if (launch_indexer(tq, ts, pa, p.D_I, p.H_I, p.fp8, true, std::min(sms, pa.total_tiles), stream) !=
-        cudaSuccess)
+    if (!cuda_ok(launch_indexer(tq, ts, pa, p.D_I, p.H_I, p.fp8, true, std::min(sms, pa.total_tiles), stream)))
       return DSA_ERR_CUDA;
   }
 
@@ -208,7 +217,7 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
   sa.topk = p.topk;
   sa.fp8 = p.fp8 ? 1 : 0;
   if (!mark(ev, 1, stream)) return DSA_ERR_CUDA;
-  if (launch_threshold(sa, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!cuda_ok(launch_threshold(sa, stream))) return DSA_ERR_CUDA;
   if (!mark(ev, 2, stream)) return DSA_ERR_CUDA;
 
   IndexerArgs ea = ia;
@@ -222,13 +231,13 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
   }
   if (total > (1ll << 30)) return DSA_ERR_UNSUPPORTED;
   ea.total_tiles = static_cast<int>(total);
-  if (launch_indexer(tq, tk, ea, p.D_I, p.H_I, p.fp8, false, static_cast<int>(std::min<long long>(sms, total)),
-                     stream) != cudaSuccess)
+  if (!cuda_ok(launch_indexer(tq, tk, ea, p.D_I, p.H_I, p.fp8, false,
+                              static_cast<int>(std::min<long long>(sms, total)), stream)))
     return DSA_ERR_CUDA;
   if (!mark(ev, 3, stream)) return DSA_ERR_CUDA;
-  if (launch_select(sa, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!cuda_ok(launch_select(sa, stream))) return DSA_ERR_CUDA;
   if (!mark(ev, 4, stream)) return DSA_ERR_CUDA;
-  if (launch_fallback(sa, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!cuda_ok(launch_fallback(sa, stream))) return DSA_ERR_CUDA;
   if (!mark(ev, 5, stream)) return DSA_ERR_CUDA;
   return DSA_OK;
 }
@@ -281,7 +290,7 @@ dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, unsigned 
   a.t0 = t0;
   a.Lq = Lq;
   a.scale_log2 = p.scale * 1.4426950408889634f;
-  return launch_sparse_mla(tq, a, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  return cuda_ok(launch_sparse_mla(tq, a, stream)) ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // namespace
@@ -289,6 +298,10 @@ dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, unsigned 
 extern "C" {
 
 int dsa_version(void) { return 1; }
+
+const char *dsa_last_error_string(void) {
+  return t_last_cuda_error == cudaSuccess ? "no CUDA error recorded" : cudaGetErrorString(t_last_cuda_error);
+}
 
 const char *dsa_status_string(dsa_status_t s) {
   switch (s) {
@@ -322,7 +335,7 @@ dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float 
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   CUtensorMap tq, tk;
   if (!make_indexer_maps(p, &tq, &tk)) return DSA_ERR_CUDA;
-  if (cudaMemsetAsync(ws.status, 0, kHeaderBytes, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!cuda_ok(cudaMemsetAsync(ws.status, 0, kHeaderBytes, stream))) return DSA_ERR_CUDA;
   for (int t0 = 0; t0 < L; t0 += QB) {
     st = run_indexer_block(p, tq, tk, ws, t0, std::min(QB, L - t0), stream);
     if (st != DSA_OK) return st;
@@ -346,7 +359,7 @@ dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, const int32_t
   CUtensorMap tq;
   if (!make_mla_maps(p, &tq)) return DSA_ERR_CUDA;
   unsigned *status = static_cast<unsigned *>(workspace);
-  if (cudaMemsetAsync(status, 0, kHeaderBytes, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!cuda_ok(cudaMemsetAsync(status, 0, kHeaderBytes, stream))) return DSA_ERR_CUDA;
   return run_mla_block(p, tq, status, 0, L, stream);
 }
 
@@ -395,7 +408,7 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, const floa
   if (!make_indexer_maps(ip, &tq, &tk) || !make_mla_maps(mp, &mq)) return DSA_ERR_CUDA;
   const int nblocks = (L + QB - 1) / QB;
   if (events != nullptr && n_events < 7 * nblocks) return DSA_ERR_INVALID_ARG;
-  if (cudaMemsetAsync(ws.status, 0, kHeaderBytes, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!cuda_ok(cudaMemsetAsync(ws.status, 0, kHeaderBytes, stream))) return DSA_ERR_CUDA;
   for (int t0 = 0; t0 < L; t0 += QB) {
     const int Lb = std::min(QB, L - t0);
     cudaEvent_t *ev = events ? events + 7 * (t0 / QB) : nullptr;
@@ -442,8 +455,8 @@ dsa_status_t dsa_workspace_status(const void *workspace, dsa_stream_t stream_, u
   if (workspace == nullptr || flags == nullptr) return DSA_ERR_INVALID_ARG;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   unsigned v = 0;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return DSA_ERR_CUDA;
-  if (cudaMemcpy(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!cuda_ok(cudaStreamSynchronize(stream))) return DSA_ERR_CUDA;
+  if (!cuda_ok(cudaMemcpy(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost))) return DSA_ERR_CUDA;
   *flags = v;
   return v == 0 ? DSA_OK : DSA_ERR_INTERNAL;
 }

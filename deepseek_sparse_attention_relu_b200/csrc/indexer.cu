@@ -19,8 +19,8 @@
 // 256 / H_I queries x H_I heads = 256 rows x D_I (UMMA N = 256), K = D_I.
 // Each TMEM lane then holds one key and each epilogue thread reduces the heads
 // of its key locally.  Warp roles: warp 0 TMA producer, warp 1 MMA issuer and
-// TMEM owner, warps 2..9 epilogue (two per TMEM lane quarter, each pair
-// splitting the 256 accumulator columns).  The accumulator is double-buffered
+// TMEM owner, warps 2..17 epilogue (four per TMEM lane quarter, each taking 64
+// of the 256 accumulator columns).  The accumulator is double-buffered
 // (2 x 256 columns) so the epilogue of tile i overlaps the MMA of tile i+1.
 #include <cuda_runtime.h>
 
@@ -42,22 +42,23 @@ struct IdxCfg {
   static constexpr int QG = BN / HI;
   static constexpr int K_TILE = BM * ROW_BYTES;
   static constexpr int Q_TILE = BN * ROW_BYTES;
-  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_WARPS = 16;                   // four per TMEM lane quarter
   static constexpr int THREADS = 64 + EPI_WARPS * 32;
-  static constexpr int QH = QG / 2;                       // queries per epilogue warp
-  static constexpr int SB = (256 / QH) < 32 ? 32 : (256 / QH);  // staged candidates per (warp, query)
+  static constexpr int COLS = BN / 4;                     // accumulator columns per epilogue warp
+  static constexpr int QH = QG / 4;                       // queries per epilogue warp
+  static constexpr int SB = (128 / QH) < 32 ? 32 : (128 / QH);  // staged candidates per (warp, query)
   static constexpr int STG_BYTES = EPI_WARPS * QH * SB * 8;
   static constexpr int SMEM_BUDGET = 224 * 1024;
-  static constexpr int FIXED = Q_TILE + STG_BYTES + 2 * EPI_WARPS * 128 * 4 + 2048;
+  static constexpr int FIXED = Q_TILE + STG_BYTES + 2 * EPI_WARPS * COLS * 4 + 2048;
   static constexpr int STAGES_FIT = (SMEM_BUDGET - FIXED) / K_TILE;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   // shared memory carve-up (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_TILE;
   static constexpr int OFF_STG = OFF_K + STAGES * K_TILE;        // [EPI_WARPS][QH][SB] candidate keys
-  static constexpr int OFF_W = OFF_STG + STG_BYTES;              // [EPI_WARPS][128] floats
-  static constexpr int OFF_TAU = OFF_W + EPI_WARPS * 128 * 4;    // [EPI_WARPS][QH] float thresholds
-  static constexpr int OFF_BAR = OFF_TAU + EPI_WARPS * 128 * 4;  // mbarriers
+  static constexpr int OFF_W = OFF_STG + STG_BYTES;               // [EPI_WARPS][COLS] floats
+  static constexpr int OFF_TAU = OFF_W + EPI_WARPS * COLS * 4;    // [EPI_WARPS][QH] float thresholds
+  static constexpr int OFF_BAR = OFF_TAU + EPI_WARPS * COLS * 4;  // mbarriers
   static constexpr int NBAR = 2 * STAGES + 2 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // tmem addr, abort flag, counters
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
@@ -66,7 +67,7 @@ struct IdxCfg {
   static_assert(ROW_BYTES % 128 == 0, "indexer rows must be whole 128-byte atoms");
   static_assert(HI % 4 == 0, "head weights are read four at a time");
   static_assert(QG * HI == BN, "H_I must divide 256");
-  static_assert((QG / 2) * HI == 128, "each epilogue half covers 128 columns");
+  static_assert(QH * HI == COLS && COLS % 32 == 0, "each epilogue warp covers whole queries");
 };
 
 union F2U {
@@ -255,14 +256,15 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
       const bool last_of_group = (nx.left == 0) || (nx.g != g);
       if (lane == 0) {
         const unsigned d_tmem = tmem_base + acc * 256;
-        const unsigned a_base = smem_u32(k_s + stage * C::K_TILE);
-        const unsigned b_base = smem_u32(q_s);
+        const uint64_t a0 = smem_desc_sw128(smem_u32(k_s + stage * C::K_TILE), 16, 1024);
+        const uint64_t b0 = smem_desc_sw128(smem_u32(q_s), 16, 1024);
 #pragma unroll
         for (int at = 0; at < C::ATOMS; ++at) {
 #pragma unroll
           for (int ks = 0; ks < C::KSTEPS_PER_ATOM; ++ks) {
-            const uint64_t ad = smem_desc_sw128(a_base + at * C::BM * 128 + ks * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(b_base + at * C::BN * 128 + ks * 32, 16, 1024);
+            // offsets go into the start-address field (address >> 4), which cannot carry
+            const uint64_t ad = a0 + static_cast<uint64_t>((at * C::BM * 128 + ks * 32) >> 4);
+            const uint64_t bd = b0 + static_cast<uint64_t>((at * C::BN * 128 + ks * 32) >> 4);
             const unsigned accum = (at | ks) ? 1u : 0u;
             if (FP8)
               mma_fp8_ss(d_tmem, ad, bd, idesc, accum);
@@ -293,9 +295,9 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;          // 0..7
+    const int ew = warp - 2;          // 0..15
     const int quarter = warp & 3;     // TMEM lane quarter this warp may access
-    const int half = ew >> 2;         // which 128 accumulator columns
+    const int slot = ew >> 2;         // which 64 accumulator columns
     constexpr int QH = C::QH;         // queries per warp
     constexpr int SB = C::SB;
     TileCursor c = idx_cursor_begin(a, C::QG);
@@ -303,8 +305,8 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     unsigned acc_phase = 0;
     bool ok = true;
     const unsigned lane_mask_lt = (1u << lane) - 1u;
-    float *w_w = w_s + ew * 128;   // this warp's head weights: [QH queries][HI]
-    float *tau_w = tau_s + ew * 128;
+    float *w_w = w_s + ew * C::COLS;   // this warp's head weights: [QH queries][HI]
+    float *tau_w = tau_s + ew * C::COLS;
     unsigned long long *stg = reinterpret_cast<unsigned long long *>(smem + C::OFF_STG) + ew * QH * SB;
     int cnt[QH];                   // staged candidates per query (warp-uniform)
 #pragma unroll
@@ -314,7 +316,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     auto flush = [&](int qq, int gq) {
       const int n = cnt[qq];
       if (n == 0) return;
-      const int tl = gq * C::QG + half * QH + qq;
+      const int tl = gq * C::QG + slot * QH + qq;
       __syncwarp();
       int base = 0;
       if (lane == 0) base = atomicAdd(&a.cand_count[tl], n);
@@ -337,13 +339,13 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
         // Each warp stages the head weights / thresholds of its own queries
         // (no cross-warp barrier, so an aborting warp cannot strand the others).
         __syncwarp();
-        for (int j = lane; j < 128; j += 32) {
-          const int tl = g * C::QG + half * QH + j / HI;
-          w_w[j] = (tl < a.Lb) ? a.w[static_cast<long long>(g * C::QG + half * QH) * HI + j] : 0.0f;
+        for (int j = lane; j < C::COLS; j += 32) {
+          const int tl = g * C::QG + slot * QH + j / HI;
+          w_w[j] = (tl < a.Lb) ? a.w[static_cast<long long>(g * C::QG + slot * QH) * HI + j] : 0.0f;
         }
         if (!PILOT) {
           for (int j = lane; j < QH; j += 32) {
-            const int tl = g * C::QG + half * QH + j;
+            const int tl = g * C::QG + slot * QH + j;
             tau_w[j] = (tl < a.Lb) ? threshold_float(a.tau[tl]) : INFINITY;
           }
         }
@@ -352,10 +354,11 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
       }
       if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      uint32_t v[4][32];
-      const unsigned taddr = tmem_base + (static_cast<unsigned>(quarter * 32) << 16) + acc * 256 + half * 128;
+      uint32_t v[C::COLS / 32][32];
+      const unsigned taddr =
+          tmem_base + (static_cast<unsigned>(quarter * 32) << 16) + acc * 256 + slot * C::COLS;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_ld_32x32b_x32(taddr + ch * 32, v[ch]);
+      for (int ch = 0; ch < C::COLS / 32; ++ch) tmem_ld_32x32b_x32(taddr + ch * 32, v[ch]);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
       const int key = c.tile * C::BM + quarter * 32 + lane;
 #pragma unroll
       for (int qq = 0; qq < QH; ++qq) {
-        const int tl = g * C::QG + half * QH + qq;  // query within the block
+        const int tl = g * C::QG + slot * QH + qq;  // query within the block
         const float4 *wq = reinterpret_cast<const float4 *>(w_w + qq * HI);
         float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
 #pragma unroll

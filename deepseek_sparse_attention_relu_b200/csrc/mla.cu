@@ -182,18 +182,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr unsigned idesc_qk = make_idesc(HT, BK, 1u, 0u, 0u);   // S = Q K^T, both K-major
     constexpr unsigned idesc_pv = make_idesc(HT, 256, 1u, 0u, 1u);  // O += P V, V MN-major
     bool ok = mbar_wait(q_full, 0u, abort_flag);
-    const unsigned q_base = smem_u32(q_s);
-    const unsigned p_base = smem_u32(p_s);
+    // Descriptors are built once; an operand offset is added to the start
+    // address field (address >> 4; shared addresses stay below 2^18, so the
+    // 14-bit field never carries).
+    const uint64_t q_desc = smem_desc_sw128(smem_u32(q_s), 16, 1024);
+    const uint64_t p_desc = smem_desc_sw128(smem_u32(p_s), 16, 1024);
+    const uint64_t k_desc[2] = {smem_desc_sw128(smem_u32(kv_s), 16, 1024),
+                                smem_desc_sw128(smem_u32(kv_s + KV_BYTES), 16, 1024)};
+    const uint64_t v_desc[2] = {smem_desc_sw128(smem_u32(kv_s), ATOM_BYTES, 1024),
+                                smem_desc_sw128(smem_u32(kv_s + KV_BYTES), ATOM_BYTES, 1024)};
     auto issue_pv = [&](int jj) {
-      const unsigned v_base = smem_u32(kv_s + (jj & 1) * KV_BYTES);
+      const uint64_t vd = v_desc[jj & 1];
 #pragma unroll
       for (int ks = 0; ks < BK / 16; ++ks) {
-        const uint64_t pd = smem_desc_sw128(p_base + ks * 32, 16, 1024);
-        const uint64_t vlo = smem_desc_sw128(v_base + ks * 2048, ATOM_BYTES, 1024);
-        const uint64_t vhi = smem_desc_sw128(v_base + 4 * ATOM_BYTES + ks * 2048, ATOM_BYTES, 1024);
         const unsigned acc = (jj > 0 || ks > 0) ? 1u : 0u;
-        mma_bf16_ss(o_lo, pd, vlo, idesc_pv, acc);
-        mma_bf16_ss(o_hi, pd, vhi, idesc_pv, acc);
+        mma_bf16_ss(o_lo, p_desc + ((ks * 32) >> 4), vd + ((ks * 2048) >> 4), idesc_pv, acc);
+        mma_bf16_ss(o_hi, p_desc + ((ks * 32) >> 4), vd + ((4 * ATOM_BYTES + ks * 2048) >> 4), idesc_pv, acc);
       }
       tc_commit(&kv_empty[jj & 1]);
       tc_commit(p_free);
@@ -225,13 +229,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         if (lane == 0) {
           const int st = nq & 1;
-          const unsigned k_base = smem_u32(kv_s + st * KV_BYTES);
+          const uint64_t kd = k_desc[st];
+          const unsigned s_tmem = s_col + st * 64;
+#pragma unroll
           for (int at = 0; at < ATOMS; ++at) {
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t qd = smem_desc_sw128(q_base + at * ATOM_BYTES + ks * 32, 16, 1024);
-              const uint64_t kd = smem_desc_sw128(k_base + at * ATOM_BYTES + ks * 32, 16, 1024);
-              mma_bf16_ss(s_col + st * 64, qd, kd, idesc_qk, (at | ks) ? 1u : 0u);
+              const uint64_t off = static_cast<uint64_t>((at * ATOM_BYTES + ks * 32) >> 4);
+              mma_bf16_ss(s_tmem, q_desc + off, kd + off, idesc_qk, (at | ks) ? 1u : 0u);
             }
           }
           tc_commit(&s_full[st]);

@@ -68,6 +68,10 @@ int dsa_version(void);
 /* Human-readable name of a status code (static string, never NULL). */
 const char *dsa_status_string(dsa_status_t status);
 
+/* Message of the CUDA error behind the calling thread's most recent
+ * DSA_ERR_CUDA (static string, never NULL; "no CUDA error recorded" if none). */
+const char *dsa_last_error_string(void);
+
 /*
  * Workspace (bytes) that dsa_indexer_topk needs for these sizes.  A larger
  * buffer is fine.  A smaller one that still holds the fixed part shrinks the
