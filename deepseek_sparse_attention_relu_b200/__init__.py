@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 
 EXPORTED = ("dsa_version", "dsa_status_string", "dsa_last_error_string", "dsa_indexer_topk_workspace", "dsa_indexer_topk",
             "dsa_sparse_mla_workspace", "dsa_sparse_mla_prefill", "dsa_prefill_chunk_workspace",
-            "dsa_prefill_chunk", "dsa_prefill_chunk_profiled", "dsa_workspace_status")
+            "dsa_prefill_chunk", "dsa_prefill_chunk_profiled", "dsa_workspace_status",
+            "dsa_indexer_topk_noalloc")
 
 _lib = None
 
@@ -69,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_prefill_chunk.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, I, P, P, P, P, Z, P]
         L.dsa_prefill_chunk_profiled.restype = I
         L.dsa_prefill_chunk_profiled.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, I, P, P, P, P, Z, P, P, I]
+        L.dsa_indexer_topk_noalloc.restype = I
+        L.dsa_indexer_topk_noalloc.argtypes = [P, P, P, I, I, I, I, I, I, I, P, P, P]
         L.dsa_workspace_status.restype = I
         L.dsa_workspace_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint)]
         _lib = L
@@ -147,6 +150,26 @@ def dsa_indexer_topk(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, 
         topk, _dev(topk_idx, "topk_idx", (torch.int32,)), _dev(topk_score, "topk_score", (torch.float32,)),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)),
         "dsa_indexer_topk")
+
+
+def dsa_indexer_topk_noalloc(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, q_pos0: int, topk: int,
+                             topk_idx: torch.Tensor, topk_score: torch.Tensor | None = None, stream=None) -> None:
+    """dsa_indexer_topk without a workspace, for callers that cannot allocate device memory (inside CUDA graph
+    capture, under a runtime that plans all memory up front, or on a fully reserved device).  The scratch is a
+    fixed 16 MiB array inside libdsa.so shared by every call on the device: calls that overlap on the GPU race,
+    and problems too large for it raise DSAError(DSA_ERR_WORKSPACE).  The first call on a device looks up the
+    array's address, so make it before any stream capture."""
+    L, H_I, D_I = q_idx.shape
+    N = k_idx.shape[0]
+    dt = _dtype_code(q_idx)
+    if k_idx.dtype != q_idx.dtype or k_idx.shape[1] != D_I or tuple(w.shape) != (L, H_I):
+        raise ValueError("inconsistent indexer operand shapes or dtypes")
+    if tuple(topk_idx.shape) != (L, topk):
+        raise ValueError("topk_idx must be [L, topk]")
+    _check(lib().dsa_indexer_topk_noalloc(
+        _dev(q_idx, "q_idx"), _dev(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt, L, N, H_I, D_I, q_pos0,
+        topk, _dev(topk_idx, "topk_idx", (torch.int32,)), _dev(topk_score, "topk_score", (torch.float32,)),
+        _stream(stream)), "dsa_indexer_topk_noalloc")
 
 
 def dsa_sparse_mla_prefill(q: torch.Tensor, kv: torch.Tensor, topk_idx: torch.Tensor, scale: float,

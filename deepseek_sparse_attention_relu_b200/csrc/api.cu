@@ -462,3 +462,71 @@ dsa_status_t dsa_workspace_status(const void *workspace, dsa_stream_t stream_, u
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// dsa_indexer_topk_noalloc: the indexer top-k for callers that cannot allocate
+// device memory (see include/dsa.h).  Its scratch is this file-scope device
+// array, held by every GPU that loads the library until the process exits.
+// Host code cannot use the array's name as a device address: the address is
+// looked up once per device with cudaGetSymbolAddress and passed on.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+constexpr int kNoAllocQueryBlock = 64;                      // queries per block in the fixed scratch
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void *g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device; the first call
+// per device does the lookup.
+dsa_status_t noalloc_scratch(void **out) {
+  int dev = 0;
+  if (!cuda_ok(cudaGetDevice(&dev))) return DSA_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return DSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (!cuda_ok(cudaGetSymbolAddress(&p, g_noalloc_scratch))) return DSA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" dsa_status_t dsa_indexer_topk_noalloc(const void *q_idx, const void *k_idx, const float *w,
+                                                 dsa_dtype_t dtype, int L, int N, int H_I, int D_I, int q_pos0,
+                                                 int topk, int32_t *topk_idx, float *topk_score,
+                                                 dsa_stream_t stream_) {
+  if (dtype != DSA_BF16 && dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID_ARG;
+  IndexerProblem p{q_idx, k_idx, w, dtype == DSA_FP8_E4M3, L, N, H_I, D_I, q_pos0, topk, topk_idx, topk_score};
+  dsa_status_t st = check_indexer_args(p);
+  if (st != DSA_OK) return st;
+  const int QB = std::min(L, kNoAllocQueryBlock);
+  // Too large for the fixed scratch: refuse before touching the device.
+  if (idx_fixed_bytes(QB, N) + static_cast<size_t>(QB) * default_cap(topk) * 8 > kNoAllocScratchBytes)
+    return DSA_ERR_WORKSPACE;
+  void *scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != DSA_OK) return st;
+  IdxWorkspace ws;
+  if (!carve_idx_ws(scratch, kNoAllocScratchBytes, QB, N, &ws)) return DSA_ERR_WORKSPACE;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  CUtensorMap tq, tk;
+  if (!make_indexer_maps(p, &tq, &tk)) return DSA_ERR_CUDA;
+  // The array keeps the previous call's contents: clear the status word and
+  // the fallback counters; every other region is rewritten before it is read.
+  if (!cuda_ok(cudaMemsetAsync(ws.status, 0, kHeaderBytes, stream))) return DSA_ERR_CUDA;
+  for (int t0 = 0; t0 < L; t0 += QB) {
+    st = run_indexer_block(p, tq, tk, ws, t0, std::min(QB, L - t0), stream);
+    if (st != DSA_OK) return st;
+  }
+  return DSA_OK;
+}

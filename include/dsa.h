@@ -101,6 +101,31 @@ dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float 
                               int N, int H_I, int D_I, int q_pos0, int topk, int32_t *topk_idx, float *topk_score,
                               void *workspace, size_t workspace_bytes, dsa_stream_t stream);
 
+/*
+ * dsa_indexer_topk for callers that cannot allocate device memory: code that
+ * runs inside a CUDA graph being captured or replayed, code that owns no
+ * allocator (an inference runtime whose memory is planned once up front), or
+ * a process whose device memory is already fully reserved.  Same arguments
+ * and results as dsa_indexer_topk, minus the workspace: the scratch is one
+ * fixed 16 MiB device array inside libdsa.so (every GPU that loads the library
+ * holds it until the process exits).  The pages describe no counterpart; this
+ * is a property of this library only.
+ *
+ *   - Limit: problems whose scratch exceeds 16 MiB at 64-query blocks are
+ *     rejected with DSA_ERR_WORKSPACE before anything is launched (with
+ *     top-k <= 2048 that admits N up to about 180,000 cached keys).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - No cudaMalloc or cudaFree, and no allocating library call, is made.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents; the call clears what must start at zero.  Calls that
+ *     overlap on the GPU (two streams, two host threads) race on the array
+ *     and must be serialised by the caller.
+ */
+dsa_status_t dsa_indexer_topk_noalloc(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
+                                      int L, int N, int H_I, int D_I, int q_pos0, int topk, int32_t *topk_idx,
+                                      float *topk_score, dsa_stream_t stream);
+
 /* Workspace (bytes) for dsa_sparse_mla_prefill: the status word only. */
 size_t dsa_sparse_mla_workspace(int L, int H, int topk);
 
