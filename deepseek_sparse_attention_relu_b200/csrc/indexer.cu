@@ -354,19 +354,24 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
       }
       if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      uint32_t v[C::COLS / 32][32];
       const unsigned taddr =
           tmem_base + (static_cast<unsigned>(quarter * 32) << 16) + acc * 256 + slot * C::COLS;
-#pragma unroll
-      for (int ch = 0; ch < C::COLS / 32; ++ch) tmem_ld_32x32b_x32(taddr + ch * 32, v[ch]);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
-
       const int key = c.tile * C::BM + quarter * 32 + lane;
+      // One 32-column chunk of the accumulator at a time (keeps the live
+      // register set small); the buffer goes back to the MMA warp after the
+      // last chunk has been read.
 #pragma unroll
-      for (int qq = 0; qq < QH; ++qq) {
+      for (int ch = 0; ch < C::COLS / 32; ++ch) {
+      uint32_t vc[32];
+      tmem_ld_32x32b_x32(taddr + ch * 32, vc);
+      tmem_ld_wait();
+      if (ch == C::COLS / 32 - 1) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      }
+#pragma unroll
+      for (int qq = ch * 32 / HI; qq < (ch + 1) * 32 / HI; ++qq) {
         const int tl = g * C::QG + slot * QH + qq;  // query within the block
         const float4 *wq = reinterpret_cast<const float4 *>(w_w + qq * HI);
         float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
@@ -374,10 +379,10 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
         for (int h4 = 0; h4 < HI / 4; ++h4) {
           const float4 w4 = wq[h4];
           const int col = qq * HI + 4 * h4;
-          const float r0 = fmaxf(__uint_as_float(v[(col + 0) / 32][(col + 0) % 32]), 0.0f);
-          const float r1 = fmaxf(__uint_as_float(v[(col + 1) / 32][(col + 1) % 32]), 0.0f);
-          const float r2 = fmaxf(__uint_as_float(v[(col + 2) / 32][(col + 2) % 32]), 0.0f);
-          const float r3 = fmaxf(__uint_as_float(v[(col + 3) / 32][(col + 3) % 32]), 0.0f);
+          const float r0 = fmaxf(__uint_as_float(vc[(col + 0) % 32]), 0.0f);
+          const float r1 = fmaxf(__uint_as_float(vc[(col + 1) % 32]), 0.0f);
+          const float r2 = fmaxf(__uint_as_float(vc[(col + 2) % 32]), 0.0f);
+          const float r3 = fmaxf(__uint_as_float(vc[(col + 3) % 32]), 0.0f);
           acc0 = ffma2(make_float2(w4.x, w4.y), make_float2(r0, r1), acc0);
           acc1 = ffma2(make_float2(w4.z, w4.w), make_float2(r2, r3), acc1);
         }
@@ -398,6 +403,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
             cnt[qq] += n;
           }
         }
+      }
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       idx_cursor_next(c, a, C::QG);

@@ -16,9 +16,9 @@
 //     layout; a tensor-map gather (tile::gather4) was measured to issue too
 //     slowly for 1,152-byte rows;
 //   * S = Q K^T on tcgen05 (M = 64 heads, N = 64 keys, K = 576), fp32 in TMEM;
-//   * softmax warps read S from TMEM, keep a running max (rescaling the output
-//     only when the max grows by more than 2^8) and write P (bf16) to shared
-//     memory in the UMMA layout;
+//   * softmax warps read S from TMEM (two lanes per head row, 32 key columns
+//     each), keep a running max (rescaling the output only when the max grows
+//     by more than 2^8) and write P (bf16) to shared memory in the UMMA layout;
 //   * O += P V on tcgen05 (M = 64, N = 2 x 256 latent columns, K = 64 keys),
 //     V read in place from the gathered tile as an MN-major operand.
 // TMEM: the two 64 x 256 fp32 halves of O sit in the two half-subpartitions
@@ -269,26 +269,26 @@ __global__ void __launch_bounds__(THREADS, 1)
     const unsigned lane_base = static_cast<unsigned>(quarter * 32) << 16;
     float m_used = -INFINITY, l = 0.0f, l_exact = 0.0f;  // l: sum of the bf16 P used; l_exact: fp32 sum for the LSE
     bool ok = true;
+    const int c0 = (lane >> 4) * 32;  // this thread's 32 of the tile's 64 key columns
     for (int j = 0; j < ntiles; ++j) {
       const int sb = j & 1;
       if (!mbar_wait(&s_full[sb], (j >> 1) & 1u, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sv[2][32];
-      tmem_ld_32x32b_x32(s_col + lane_base + sb * 64, sv[0]);
-      tmem_ld_32x32b_x32(s_col + lane_base + sb * 64 + 32, sv[1]);
+      uint32_t sv[32];
+      tmem_ld_16x32bx2_x32(s_col + lane_base + sb * 64, sv);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[sb]);
-      const unsigned long long vmask = valid_s[j & 1];
-      float z[64];
+      const unsigned vbits = static_cast<unsigned>(valid_s[j & 1] >> c0);
+      float z[32];
       float tmax = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const bool v = (vmask >> c) & 1ull;
-        z[c] = v ? __uint_as_float(sv[c >> 5][c & 31]) * a.scale_log2 : -INFINITY;
+      for (int c = 0; c < 32; ++c) {
+        z[c] = ((vbits >> c) & 1u) ? __uint_as_float(sv[c]) * a.scale_log2 : -INFINITY;
         tmax = fmaxf(tmax, z[c]);
       }
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));  // whole row (both halves)
       const float m_old = m_used;
       bool rescale = false;
       if (tmax > m_used + kRescaleLog2 || (m_used == -INFINITY && tmax > -INFINITY)) {
@@ -296,10 +296,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         m_used = tmax;
       }
       // P in bf16, rounded once; the normaliser sums the rounded values.
-      uint32_t pk[32];
+      uint32_t pk[16];
       float tsum = 0.0f, tsum_exact = 0.0f;
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
+      for (int c = 0; c < 32; c += 2) {
         const float p0 = (m_used == -INFINITY) ? 0.0f : fast_exp2(z[c] - m_used);
         const float p1 = (m_used == -INFINITY) ? 0.0f : fast_exp2(z[c + 1] - m_used);
         const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
@@ -308,6 +308,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         tsum_exact += p0 + p1;
         pk[c >> 1] = *reinterpret_cast<const uint32_t *>(&b);
       }
+      tsum += __shfl_xor_sync(0xffffffffu, tsum, 16);
+      tsum_exact += __shfl_xor_sync(0xffffffffu, tsum_exact, 16);
       const float alpha = rescale ? fast_exp2(m_old - m_used) : 1.0f;
       l = l * alpha + tsum;
       l_exact = l_exact * alpha + tsum_exact;
@@ -315,33 +317,30 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait(p_free, (j - 1) & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
       }
-      // Rescale O (both halves) when the running max moved: lanes 0-15 own the
-      // O_lo rows, lanes 16-31 the O_hi rows of the same heads.
-      const bool any_rescale = __any_sync(0xffffffffu, rescale && lane < 16);
-      if (any_rescale) {
-        const float my_alpha = __shfl_sync(0xffffffffu, alpha, r16);
-        const bool mine = __shfl_sync(0xffffffffu, rescale ? 1 : 0, r16) != 0;
-        // One 32x32b access covers lanes 32q..32q+31: O_lo rows then O_hi rows.
-        const unsigned obase = o_lo + lane_base;
+      // Rescale O when the running max moved: lanes 0-15 own the O_lo rows and
+      // lanes 16-31 the O_hi rows of the same heads (same alpha).
+      if (__any_sync(0xffffffffu, rescale)) {
+        const unsigned obase = o_lo + lane_base;  // one 32x32b access: O_lo rows then O_hi rows
 #pragma unroll 1
         for (int ch = 0; ch < 8; ++ch) {
           uint32_t ov[32];
           tmem_ld_32x32b_x32(obase + ch * 32, ov);
           tmem_ld_wait();
-          if (mine) {
+          if (rescale) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * my_alpha);
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
           }
           tmem_st_32x32b_x32(obase + ch * 32, ov);
         }
         tmem_st_wait();
       }
-      if (lane < 16) {
+      {
         uint8_t *prow = p_s + row * 128;
+        const int cbase = c0 >> 3;  // first 16-byte chunk of this thread's 32 columns
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
+        for (int ch = 0; ch < 4; ++ch) {
           const uint4 v = make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-          *reinterpret_cast<uint4 *>(prow + ((ch ^ (row & 7)) << 4)) = v;
+          *reinterpret_cast<uint4 *>(prow + (((cbase + ch) ^ (row & 7)) << 4)) = v;
         }
       }
       fence_proxy_async_smem();
@@ -355,8 +354,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       *abort_flag = 1;
     } else {
       tc_fence_after();
-      const float l_row = __shfl_sync(0xffffffffu, l, r16);
-      const float inv = l_row > 0.0f ? 1.0f / l_row : 0.0f;
+      const float inv = l > 0.0f ? 1.0f / l : 0.0f;  // both halves of a row hold the row's l
       const int head = hg * HT + row;
       const int dim0 = lane < 16 ? 0 : 256;
       uint16_t *orow = a.out + (static_cast<long long>(t) * a.H + head) * LAT + dim0;

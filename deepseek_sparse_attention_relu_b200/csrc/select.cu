@@ -88,9 +88,12 @@ __device__ void block_radix_select(Fetch fetch, int n, int need, KeyT &prefix_ou
 }
 
 // ------------------------------------------------------------------ threshold
+constexpr int kMaxSamples = 4096;
+
 __global__ void __launch_bounds__(256) threshold_kernel(SelectArgs a) {
   __shared__ unsigned hist[256];
   __shared__ unsigned misc[4];
+  __shared__ unsigned keys[kMaxSamples];  // the query's sample scores as order-preserving keys
   const int tl = blockIdx.x;
   if (threadIdx.x == 0) {
     a.cand_count[tl] = 0;
@@ -110,9 +113,10 @@ __global__ void __launch_bounds__(256) threshold_kernel(SelectArgs a) {
     if (rd < a.n_samples) {
       const int r = static_cast<int>(rd);
       const float *row = a.dense + static_cast<long long>(tl) * a.dense_ld;
+      for (int i = threadIdx.x; i < a.n_samples; i += blockDim.x) keys[i] = float_order_key(row[i]);
+      __syncthreads();
       unsigned prefix, mask;
-      block_radix_select<unsigned>([&](int i) { return float_order_key(row[i]); }, a.n_samples, r, prefix, mask,
-                                   hist, misc);
+      block_radix_select<unsigned>([&](int i) { return keys[i]; }, a.n_samples, r, prefix, mask, hist, misc);
       tau = prefix;
     }
   }
@@ -140,11 +144,43 @@ __device__ void block_bitonic_sort(unsigned long long *v, int n) {
 }
 
 // ------------------------------------------------------------------ select
+constexpr int kSmemCand = 8192;        // candidates staged in shared memory (larger lists stay in L2)
+constexpr int kBitmapKeys = 262144;    // ascending output through a shared bitmap up to this many keys
+
+// Exclusive prefix sum of one int per thread over the block (blockDim.x <= 1024).
+__device__ int block_exclusive_scan(int v, int *warp_tot, int *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = (blockDim.x + 31) >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < nwarps ? warp_tot[lane] : 0;
+    int ti = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, ti, off);
+      if (lane >= off) ti += o;
+    }
+    if (lane < nwarps) warp_tot[lane] = ti - t;
+    if (lane == 31) *total = ti;
+  }
+  __syncthreads();
+  return warp_tot[warp] + incl - v;
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
+  extern __shared__ __align__(16) unsigned char sel_smem[];
+  unsigned long long *cs = reinterpret_cast<unsigned long long *>(sel_smem);         // staged candidates
+  unsigned char *region = sel_smem + static_cast<size_t>(min(a.cap, kSmemCand)) * 8;  // bitmap or sort buffer
   __shared__ unsigned hist[256];
   __shared__ unsigned misc[4];
-  __shared__ unsigned long long sortbuf[kMaxTopk];  // (key index << 32) | score key
-  __shared__ int nsel;
+  __shared__ int warp_tot[kSelThreads / 32];
+  __shared__ int total, nsel;
   const int tl = blockIdx.x;
   const int t = a.t0 + tl;
   const int nvis = a.q_pos0 + tl + 1;
@@ -158,17 +194,59 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     return;
   }
   const unsigned long long *cand = a.cand + static_cast<long long>(tl) * a.cap;
-  unsigned long long prefix = 0, mask = 0;
-  if (count > need) {
-    block_radix_select<unsigned long long>([&](int i) { return cand[i]; }, count, need, prefix, mask, hist, misc);
+  const bool staged = count <= kSmemCand;
+  if (staged) {
+    for (int i = threadIdx.x; i < count; i += blockDim.x) cs[i] = cand[i];
+    __syncthreads();
   }
+  auto fetch = [&](int i) { return staged ? cs[i] : cand[i]; };
+  unsigned long long prefix = 0, mask = 0;
+  if (count > need) block_radix_select<unsigned long long>(fetch, count, need, prefix, mask, hist, misc);
+  int32_t *out = a.topk_idx + static_cast<long long>(t) * a.topk;
+  float *osc = a.topk_score ? a.topk_score + static_cast<long long>(t) * a.topk : nullptr;
+
+  if (osc == nullptr && nvis <= kBitmapKeys) {
+    // Winners -> bitmap over key indices -> ordered compaction (ascending keys).
+    unsigned *bitmap = reinterpret_cast<unsigned *>(region);
+    const int nwords = (nvis + 31) >> 5;
+    for (int i = threadIdx.x; i < nwords; i += blockDim.x) bitmap[i] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < count; i += blockDim.x) {
+      const unsigned long long k = fetch(i);
+      if (k >= prefix) {
+        const unsigned idx = ~static_cast<unsigned>(k & 0xFFFFFFFFull);
+        atomicOr(&bitmap[idx >> 5], 1u << (idx & 31));
+      }
+    }
+    __syncthreads();
+    const int per = (nwords + blockDim.x - 1) / blockDim.x;
+    const int w0 = threadIdx.x * per, w1 = min(nwords, w0 + per);
+    int mine = 0;
+    for (int wd = w0; wd < w1; ++wd) mine += __popc(bitmap[wd]);
+    int pos = block_exclusive_scan(mine, warp_tot, &total);
+    for (int wd = w0; wd < w1; ++wd) {
+      unsigned bits = bitmap[wd];
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (pos < need) out[pos] = wd * 32 + b;
+        ++pos;
+      }
+    }
+    if (threadIdx.x == 0 && total != need) atomicOr(a.status, DEV_OVERFLOW);
+    for (int j = need + threadIdx.x; j < a.topk; j += blockDim.x) out[j] = -1;
+    return;
+  }
+
+  // Scores requested (or a very long cache): bitonic sort of (index, score key) pairs.
+  unsigned long long *sortbuf = reinterpret_cast<unsigned long long *>(region);
   if (threadIdx.x == 0) nsel = 0;
   int npow = 1;
   while (npow < need) npow <<= 1;
   for (int i = threadIdx.x; i < npow; i += blockDim.x) sortbuf[i] = ~0ull;
   __syncthreads();
   for (int i = threadIdx.x; i < count; i += blockDim.x) {
-    const unsigned long long k = cand[i];
+    const unsigned long long k = fetch(i);
     if (k >= prefix) {
       const int p = atomicAdd(&nsel, 1);
       const unsigned idx = ~static_cast<unsigned>(k & 0xFFFFFFFFull);
@@ -180,8 +258,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     if (threadIdx.x == 0) atomicOr(a.status, DEV_OVERFLOW);
   }
   block_bitonic_sort(sortbuf, npow);
-  int32_t *out = a.topk_idx + static_cast<long long>(t) * a.topk;
-  float *osc = a.topk_score ? a.topk_score + static_cast<long long>(t) * a.topk : nullptr;
   for (int j = threadIdx.x; j < a.topk; j += blockDim.x) {
     if (j < need) {
       const unsigned long long v = sortbuf[j];
@@ -291,7 +367,11 @@ cudaError_t launch_threshold(const SelectArgs &a, cudaStream_t stream) {
 }
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream) {
-  select_kernel<<<a.Lb, kSelThreads, 0, stream>>>(a);
+  // staged candidates + max(bitmap of kBitmapKeys bits, sort buffer of kMaxTopk pairs)
+  const int smem = min(a.cap, kSmemCand) * 8 + max(kBitmapKeys / 8, kMaxTopk * 8);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  select_kernel<<<a.Lb, kSelThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
