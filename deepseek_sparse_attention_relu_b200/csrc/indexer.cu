@@ -158,8 +158,6 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
   uint64_t *drain = q_full + 6;             // MMA drain on abort
   unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + C::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
-  int *consumed = reinterpret_cast<int *>(smem + C::OFF_MISC + 16);  // k tiles the MMA warp consumed
-  int *q_consumed = reinterpret_cast<int *>(smem + C::OFF_MISC + 20);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -177,8 +175,6 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
-    *consumed = 0;
-    *q_consumed = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -227,17 +223,21 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
         atomicOr(a.status, DEV_TIMEOUT);
         *abort_flag = 1;
       }
-      // Never leave with copies in flight: wait for every issued load to land.
-      const int done = *reinterpret_cast<volatile int *>(consumed);
-      for (int i = done; i < issued; ++i) mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1u, nullptr);
-      if (q_issued > *reinterpret_cast<volatile int *>(q_consumed))
-        mbar_wait(q_full, static_cast<unsigned>(q_issued - 1) & 1u, nullptr);
+      // Never leave with copies in flight.  Only the last STAGES issued tiles can
+      // still be landing, and each of them is the final use of its stage, so the
+      // phase parity below is unambiguous (an older phase of a reused stage would
+      // alias the current, never-completing one).
+      bool drained = true;
+      for (int i = (issued > C::STAGES ? issued - C::STAGES : 0); i < issued; ++i)
+        drained &= mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1u, nullptr);
+      if (q_issued > 0) drained &= mbar_wait(q_full, static_cast<unsigned>(q_issued - 1) & 1u, nullptr);
+      if (!drained) atomicOr(a.status, DEV_TIMEOUT);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     TileCursor c = idx_cursor_begin(a, C::QG);
     constexpr unsigned idesc = make_idesc(C::BM, C::BN, FP8 ? 0u : 1u, 0u, 0u);
-    int stage = 0, acc = 0, prev_g = -1, n = 0;
+    int stage = 0, acc = 0, prev_g = -1;
     unsigned phase = 0, acc_phase = 0, qphase = 0;
     bool ok = true;
     while (c.left > 0) {
@@ -246,7 +246,6 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
         if (!mbar_wait(q_full, qphase, abort_flag)) { ok = false; break; }
         qphase ^= 1u;
         prev_g = g;
-        if (lane == 0) *reinterpret_cast<volatile int *>(q_consumed) += 1;
       }
       if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
       if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
@@ -277,8 +276,6 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
         if (last_of_group) tc_commit(q_empty);
       }
       __syncwarp();
-      ++n;
-      if (lane == 0) *reinterpret_cast<volatile int *>(consumed) = n;
       if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       c = nx;
@@ -290,7 +287,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     // Drain: every MMA this warp issued must finish before TMEM is released.
     if (lane == 0) {
       tc_commit(drain);
-      mbar_wait(drain, 0u, nullptr);
+      if (!mbar_wait(drain, 0u, nullptr)) atomicOr(a.status, DEV_TIMEOUT);
     }
     __syncwarp();
   } else {

@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
       *abort_flag = 1;
     }
-    if (p == 0 && lane == 0) mbar_wait(q_full, 0u, nullptr);
+    if (p == 0 && lane == 0 && !mbar_wait(q_full, 0u, nullptr)) atomicOr(a.status, DEV_TIMEOUT);
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (lane == 0) {
       tc_commit(drain);
-      mbar_wait(drain, 0u, nullptr);
+      if (!mbar_wait(drain, 0u, nullptr)) atomicOr(a.status, DEV_TIMEOUT);
     }
     __syncwarp();
   } else {
