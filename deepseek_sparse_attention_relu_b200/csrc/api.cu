@@ -275,8 +275,36 @@ bool make_mla_maps(const MlaProblem &p, CUtensorMap *tq) {
                      64);
 }
 
+// ---- query packing for the attention stage (LiteDSA-style candidate reuse)
+constexpr int kPackMaxEntries = 8192;  // G * topk selection entries per pack (bounds the union)
+constexpr float kMaxUnionRatio = 0.75f; // pack when the union is at most 75% of the members' keys
+
+// Queries packed per CTA: with H <= 32 heads a 64-row tile has room for
+// 64 / H queries, and packing them over the union of their selections never
+// adds tensor work (the rows were idle) while shared keys are gathered once.
+// Capped so the attention grid still covers the GPU at least twice.
+int pack_group(int H, int topk, int Lq, int N) {
+  if (H > 32 || N > 800 * 1024) return 1;  // the pack plan's key bitmap must fit in shared memory
+  int G = 64 / H;
+  G = std::min(G, kPackMaxEntries / topk);
+  G = std::min(G, std::max(1, Lq / (2 * std::max(1, sm_count()))));
+  return std::max(G, 1);
+}
+
+// Union buffers for up to Lq queries packed G at a time (any G).
+size_t union_bytes(int Lq, int topk) {
+  // packs * (G * topk rounded up to whole 64-key tiles), for any G
+  const size_t slots = static_cast<size_t>(Lq + 64) * topk + static_cast<size_t>(Lq + 1) * 64;
+  return align256(slots * 4) + align256(slots * 8) + 3 * align256(static_cast<size_t>(Lq) * 4) + 256;
+}
+
+struct UnionWorkspace {
+  void *base = nullptr;
+  size_t bytes = 0;
+};
+
 dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, unsigned *status, int t0, int Lq,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, UnionWorkspace uw = UnionWorkspace()) {
   MlaArgs a{};
   a.topk_idx = p.topk_idx;
   a.kv = p.kv;
@@ -290,7 +318,49 @@ dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, unsigned 
   a.t0 = t0;
   a.Lq = Lq;
   a.scale_log2 = p.scale * 1.4426950408889634f;
-  return cuda_ok(launch_sparse_mla(tq, a, stream)) ? DSA_OK : DSA_ERR_CUDA;
+  a.G = 1;
+  const int G = pack_group(p.H, p.topk, Lq, p.N);
+  if (G >= 2 && uw.base != nullptr && uw.bytes >= union_bytes(Lq, p.topk)) {
+    const int npacks = (Lq + G - 1) / G;
+    const int umax = (G * p.topk + 63) / 64 * 64;  // whole 64-key tiles
+    const size_t slots = static_cast<size_t>(npacks) * umax;
+    uint8_t *b = static_cast<uint8_t *>(uw.base);
+    PackArgs pa{};
+    pa.topk_idx = p.topk_idx;
+    pa.ukeys = reinterpret_cast<int32_t *>(b);
+    pa.qmask = reinterpret_cast<unsigned long long *>(b + align256(slots * 4));
+    uint8_t *c = b + align256(slots * 4) + align256(slots * 8);
+    pa.ucount = reinterpret_cast<int *>(c);
+    pa.plist = reinterpret_cast<int *>(c + align256(static_cast<size_t>(Lq) * 4));
+    pa.slist = reinterpret_cast<int *>(c + 2 * align256(static_cast<size_t>(Lq) * 4));
+    int *counters = reinterpret_cast<int *>(c + 3 * align256(static_cast<size_t>(Lq) * 4));
+    pa.pcount = counters;
+    pa.scount = counters + 1;
+    pa.max_union_ratio = kMaxUnionRatio;
+    pa.status = status;
+    if (!cuda_ok(cudaMemsetAsync(counters, 0, 2 * sizeof(int), stream))) return DSA_ERR_CUDA;
+    pa.t0 = t0;
+    pa.Lq = Lq;
+    pa.G = G;
+    pa.topk = p.topk;
+    pa.umax = umax;
+    pa.N = p.N;
+    if (!cuda_ok(launch_pack_plan(pa, stream))) return DSA_ERR_CUDA;
+    a.G = G;
+    a.umax = umax;
+    a.ukeys = pa.ukeys;
+    a.qmask = pa.qmask;
+    a.ucount = pa.ucount;
+    a.list = pa.plist;
+    a.list_count = pa.pcount;
+    if (!cuda_ok(launch_sparse_mla(tq, a, true, stream))) return DSA_ERR_CUDA;
+    MlaArgs single = a;
+    single.G = 1;
+    single.list = pa.slist;
+    single.list_count = pa.scount;
+    return cuda_ok(launch_sparse_mla(tq, single, false, stream)) ? DSA_OK : DSA_ERR_CUDA;
+  }
+  return cuda_ok(launch_sparse_mla(tq, a, false, stream)) ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // namespace
@@ -345,7 +415,7 @@ dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float 
 
 size_t dsa_sparse_mla_workspace(int L, int H, int topk) {
   if (L <= 0 || H <= 0 || topk <= 0) return 0;
-  return kHeaderBytes;
+  return kHeaderBytes + (H <= 32 ? union_bytes(L, topk) : 0);
 }
 
 dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, const int32_t *topk_idx, int L, int N, int H,
@@ -360,7 +430,10 @@ dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, const int32_t
   if (!make_mla_maps(p, &tq)) return DSA_ERR_CUDA;
   unsigned *status = static_cast<unsigned *>(workspace);
   if (!cuda_ok(cudaMemsetAsync(status, 0, kHeaderBytes, stream))) return DSA_ERR_CUDA;
-  return run_mla_block(p, tq, status, 0, L, stream);
+  UnionWorkspace uw;
+  uw.base = static_cast<uint8_t *>(workspace) + kHeaderBytes;
+  uw.bytes = workspace_bytes - kHeaderBytes;
+  return run_mla_block(p, tq, status, 0, L, stream, uw);
 }
 
 size_t dsa_prefill_chunk_workspace(int L, int N, int H_I, int D_I, int H, int topk, int query_block,
@@ -370,6 +443,7 @@ size_t dsa_prefill_chunk_workspace(int L, int N, int H_I, int D_I, int H, int to
   const int QB = std::min(L, query_block > 0 ? query_block : kDefaultQueryBlock);
   size_t bytes = idx_fixed_bytes(QB, N) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
   if (!want_topk_out) bytes += align256(static_cast<size_t>(QB) * topk * 4);
+  if (H <= 32) bytes += union_bytes(QB, topk) + 256;
   return bytes;
 }
 
@@ -393,6 +467,17 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, const floa
     if (workspace == nullptr || workspace_bytes < need) return DSA_ERR_WORKSPACE;
     idx_bytes = (workspace_bytes - need) & ~static_cast<size_t>(255);
     block_idx = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + idx_bytes);
+  }
+  // Union buffers of the packed attention (H <= 32), below the selected keys.
+  UnionWorkspace uw;
+  if (H <= 32 && workspace != nullptr) {
+    const size_t ub = union_bytes(QB, topk);
+    if (idx_bytes >= ub + (size_t(1) << 20)) {
+      const size_t off = (idx_bytes - ub) & ~static_cast<size_t>(255);
+      uw.base = static_cast<uint8_t *>(workspace) + off;
+      uw.bytes = idx_bytes - off;
+      idx_bytes = off;
+    }
   }
   IndexerProblem ip{q_idx, k_idx, w, dtype == DSA_FP8_E4M3, L, N, H_I, D_I, q_pos0, topk,
                     topk_idx_out ? topk_idx_out : block_idx, nullptr};
@@ -421,7 +506,7 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, const floa
     }
     st = run_indexer_block(bp, tq, tk, ws, t0, Lb, stream, ev);
     if (st != DSA_OK) return st;
-    st = run_mla_block(bm, mq, ws.status, t0, Lb, stream);
+    st = run_mla_block(bm, mq, ws.status, t0, Lb, stream, uw);
     if (st != DSA_OK) return st;
     if (!mark(ev, 6, stream)) return DSA_ERR_CUDA;
   }

@@ -65,8 +65,33 @@ struct MlaArgs {
   int L, N, H, topk;
   int t0, Lq;                     // queries [t0, t0 + Lq) of the chunk in this launch
   float scale_log2;               // softmax scale * log2(e)
+  // Packed mode (G >= 2 queries of H <= 32 heads share one 64-row tile): the
+  // union of the pack's selections and, per union key, which queries chose it.
+  const int32_t *ukeys;           // [npacks, umax] ascending union keys
+  const unsigned long long *qmask;  // [npacks, umax / 64, 64]: word j of tile i = keys of tile i chosen by query j
+  const int *ucount;              // [npacks]
+  int G, umax;
+  // Optional work list: CTA i serves item list[i] (a pack in packed mode, a
+  // query in unpacked mode) and CTAs with i >= *list_count exit at once.
+  const int *list;
+  const int *list_count;
 };
 
-cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, cudaStream_t stream);
+// Union of each pack's G index rows with membership masks (packed attention).
+struct PackArgs {
+  const int32_t *topk_idx;        // [L, topk]
+  int32_t *ukeys;
+  unsigned long long *qmask;      // [npacks, umax / 64, 64] per tile and query: which keys it chose
+  int *ucount;
+  int *plist, *pcount;            // packs worth packing (union small enough)
+  int *slist, *scount;            // queries of the other packs, served one per CTA
+  unsigned *status;
+  int t0, Lq, G, topk, umax, N;
+  float max_union_ratio;          // pack when |union| <= ratio * sum of the members' selections
+};
+
+cudaError_t launch_pack_plan(const PackArgs &a, cudaStream_t stream);
+
+cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, bool packed, cudaStream_t stream);
 
 }  // namespace dsa

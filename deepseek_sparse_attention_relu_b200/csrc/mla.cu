@@ -52,7 +52,8 @@ constexpr int OFF_P = OFF_KV + STAGES * KV_BYTES;
 constexpr int OFF_BAR = OFF_P + P_BYTES;
 constexpr int NBAR = 1 + 2 * STAGES + 4 + 2 + 1;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
+constexpr int OFF_MEMB = OFF_MISC + 64;             // [STAGES][64] per-query key masks (packed mode)
+constexpr int SMEM_BYTES = OFF_MEMB + STAGES * BK * 8 + 1024;
 constexpr float kRescaleLog2 = 8.0f;
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -61,6 +62,10 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// PACKED: the CTA serves G consecutive queries of H <= 32 heads (rows
+// j*H .. j*H+H-1 of the 64-row tile belong to query j) over the union of their
+// selections; a union key counts for row r only if query r / H chose it.
+template <bool PACKED>
 __global__ void __launch_bounds__(THREADS, 1)
     sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q, MlaArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -80,12 +85,27 @@ __global__ void __launch_bounds__(THREADS, 1)
   unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
   unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + OFF_MISC + 8);  // [2]
+  unsigned long long *memb_s = reinterpret_cast<unsigned long long *>(smem + OFF_MEMB);       // [2][BK]
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int t = a.t0 + blockIdx.x;
+  int item = blockIdx.x;  // the query (or pack) this CTA serves
+  if (a.list != nullptr) {
+    if (static_cast<int>(blockIdx.x) >= *a.list_count) return;
+    item = a.list[blockIdx.x];
+  }
+  const int t = a.t0 + item * (PACKED ? a.G : 1);  // first query of this CTA
   const int hg = blockIdx.y;
-  const int ntiles = (a.topk + BK - 1) / BK;
+  const int nq = PACKED ? min(a.G, a.t0 + a.Lq - t) : 1;  // queries served
+  // Keys this CTA walks: the query's selection, or the pack's union.
+  const int nkeys = PACKED ? a.ucount[item] : a.topk;
+  const int32_t *keys = PACKED ? a.ukeys + static_cast<long long>(item) * a.umax
+                               : a.topk_idx + static_cast<long long>(t) * a.topk;
+  const unsigned long long *qmask = PACKED ? a.qmask + static_cast<long long>(item) * a.umax : nullptr;
+  const int ntiles = max(1, (nkeys + BK - 1) / BK);
+  // Output rows of the 64-row tile: global row out_row0 + r for r < row_limit.
+  const long long out_row0 = static_cast<long long>(t) * a.H + (PACKED ? 0 : hg * HT);
+  const int row_limit = PACKED ? nq * a.H : min(HT, a.H - hg * HT);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -129,22 +149,29 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int row0 = t * a.H + hg * HT;
       for (int at = 0; at < ATOMS; ++at) tma_load_2d(q_s + at * ATOM_BYTES, &tmap_q, q_full, at * 64, row0);
     }
-    const int32_t *idx_row = a.topk_idx + static_cast<long long>(t) * a.topk;
     auto load_idx = [&](int j, int (&v)[16]) {
 #pragma unroll
       for (int g = 0; g < 16; ++g) {
         const int pos = j * BK + 4 * g + r;
-        v[g] = (j < ntiles && pos < a.topk) ? idx_row[pos] : -1;
+        v[g] = (j < ntiles && pos < nkeys) ? keys[pos] : -1;
       }
     };
     const uint8_t *kv = static_cast<const uint8_t *>(a.kv);
     const unsigned stage_base = smem_u32(kv_s + p * KV_BYTES);
+    // Packed mode: lane j < G also carries query j's 64-bit key mask of the tile.
+    auto load_mask = [&](int j) -> unsigned long long {
+      return (PACKED && lane < nq && j < ntiles) ? qmask[static_cast<long long>(j) * 64 + lane] : 0ull;
+    };
     int cur[16], nxt[16];
+    unsigned long long cur_m = 0ull, nxt_m = 0ull;
     load_idx(p, cur);
+    cur_m = load_mask(p);
     for (int j = p; j < ntiles; j += 2) {
       load_idx(j + 2, nxt);
+      nxt_m = load_mask(j + 2);
       if (!mbar_wait(&kv_empty[p], ((j >> 1) & 1) ^ 1u, abort_flag)) { ok = false; break; }
       unsigned long long vbits = 0;
+      if (PACKED && lane < nq) memb_s[p * BK + lane] = cur_m;
 #pragma unroll
       for (int g = 0; g < 16; ++g) {
         const int v = cur[g];
@@ -169,6 +196,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
 #pragma unroll
       for (int g = 0; g < 16; ++g) cur[g] = nxt[g];
+      cur_m = nxt_m;
     }
     cp_async_wait_all();  // never leave with copies in flight
     if (!ok) {
@@ -280,7 +308,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[sb]);
-      const unsigned vbits = static_cast<unsigned>(valid_s[j & 1] >> c0);
+      unsigned vbits;
+      if (PACKED) {
+        // keys of this tile that the row's own query chose
+        const int qj = row / a.H;
+        vbits = qj < nq ? static_cast<unsigned>(memb_s[(j & 1) * BK + qj] >> c0) : 0u;
+      } else {
+        vbits = static_cast<unsigned>(valid_s[j & 1] >> c0);
+      }
       float z[32];
       float tmax = -INFINITY;
 #pragma unroll
@@ -355,15 +390,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
       tc_fence_after();
       const float inv = l > 0.0f ? 1.0f / l : 0.0f;  // both halves of a row hold the row's l
-      const int head = hg * HT + row;
+      const bool has_row = row < row_limit;
       const int dim0 = lane < 16 ? 0 : 256;
-      uint16_t *orow = a.out + (static_cast<long long>(t) * a.H + head) * LAT + dim0;
+      uint16_t *orow = a.out + (out_row0 + row) * LAT + dim0;
 #pragma unroll 1
       for (int ch = 0; ch < 8; ++ch) {
         uint32_t ov[32];
         tmem_ld_32x32b_x32(o_lo + lane_base + ch * 32, ov);
         tmem_ld_wait();
-        if (head < a.H) {
+        if (has_row) {
           uint32_t pkd[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -376,8 +411,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
         }
       }
-      if (lane < 16 && head < a.H && a.lse != nullptr) {
-        a.lse[static_cast<long long>(t) * a.H + head] =
+      if (lane < 16 && has_row && a.lse != nullptr) {
+        a.lse[out_row0 + row] =
             l_exact > 0.0f ? (m_used + log2f(l_exact)) * 0.69314718055994530942f : -INFINITY;
       }
     }
@@ -393,12 +428,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace mla
 
-cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(mla::sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       mla::SMEM_BYTES);
+cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, bool packed, cudaStream_t stream) {
+  auto kern = packed ? mla::sparse_mla_kernel<true> : mla::sparse_mla_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.Lq, (a.H + mla::HT - 1) / mla::HT);
-  mla::sparse_mla_kernel<<<grid, mla::THREADS, mla::SMEM_BYTES, stream>>>(tq, a);
+  dim3 grid(packed ? (a.Lq + a.G - 1) / a.G : a.Lq, packed ? 1 : (a.H + mla::HT - 1) / mla::HT);
+  kern<<<grid, mla::THREADS, mla::SMEM_BYTES, stream>>>(tq, a);
   return cudaGetLastError();
 }
 

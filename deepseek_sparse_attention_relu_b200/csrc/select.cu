@@ -361,6 +361,110 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(SelectArgs a) {
   }
 }
 
+// ------------------------------------------------------------------ pack plan
+// LiteDSA (arXiv 2607.11976, Abstract) packs neighbouring queries' candidate
+// sets for joint computation and masks each query's scores to its own set.
+// One CTA per pack of G consecutive queries: mark every selected key in a
+// shared bitmap over key indices, number the marked keys in ascending order
+// (per-word prefix popcounts give any key's rank in O(1)), and record for
+// every 64-key tile of that union which keys each query chose.  The pack is
+// packed only if the union is small enough and its rows are clean (unique,
+// in-range keys); otherwise its queries are handed to the unpacked kernel.
+constexpr int kPackThreads = 1024;
+
+__global__ void __launch_bounds__(kPackThreads) pack_plan_kernel(PackArgs a) {
+  extern __shared__ unsigned pk_words[];  // bitmap [nwords], then exclusive prefix counts [nwords]
+  __shared__ int warp_tot[kPackThreads / 32];
+  __shared__ int total, nvalid_s, bad_s;
+  __shared__ int qcount[64];
+  const int nwords = (a.N + 31) >> 5;
+  unsigned *bm = pk_words;
+  unsigned *pre = pk_words + nwords;
+  const int p = blockIdx.x;
+  const int q0 = a.t0 + p * a.G;
+  const int nq = min(a.G, a.t0 + a.Lq - q0);
+  const int n = nq * a.topk;
+  const int32_t *rows = a.topk_idx + static_cast<long long>(q0) * a.topk;
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) bm[w] = 0u;
+  if (threadIdx.x < 64) qcount[threadIdx.x] = 0;
+  if (threadIdx.x == 0) { nvalid_s = 0; bad_s = 0; }
+  __syncthreads();
+  int valid = 0, bad = 0;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int key = rows[e];
+    if (key >= 0 && key < a.N) {
+      atomicOr(&bm[key >> 5], 1u << (key & 31));
+      ++valid;
+    } else if (key != -1) {
+      ++bad;
+    }
+  }
+  if (valid) atomicAdd(&nvalid_s, valid);
+  if (bad) atomicAdd(&bad_s, bad);
+  __syncthreads();
+  const int per = (nwords + blockDim.x - 1) / blockDim.x;
+  const int w0 = threadIdx.x * per, w1 = min(nwords, w0 + per);
+  int mine = 0;
+  for (int w = w0; w < w1; ++w) mine += __popc(bm[w]);
+  int base = block_exclusive_scan(mine, warp_tot, &total);
+  for (int w = w0; w < w1; ++w) {
+    pre[w] = base;
+    base += __popc(bm[w]);
+  }
+  const int nu = min(total, a.umax);
+  const int ntiles = (nu + 63) / 64;
+  unsigned long long *qm = a.qmask + static_cast<long long>(p) * a.umax;
+  for (int i = threadIdx.x; i < ntiles * 64; i += blockDim.x) qm[i] = 0ull;
+  __syncthreads();
+  // Union keys in ascending order, and each query's membership bits.
+  int32_t *uk = a.ukeys + static_cast<long long>(p) * a.umax;
+  for (int w = w0; w < w1; ++w) {
+    unsigned bits = bm[w];
+    int u = pre[w];
+    while (bits) {
+      const int b = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (u < a.umax) uk[u] = w * 32 + b;
+      ++u;
+    }
+  }
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int key = rows[e];
+    if (key < 0 || key >= a.N) continue;
+    const int j = e / a.topk;
+    const int u = pre[key >> 5] + __popc(bm[key >> 5] & ((1u << (key & 31)) - 1u));
+    if (u < a.umax) {
+      const unsigned long long bit = 1ull << (u & 63);
+      const unsigned long long old = atomicOr(&qm[(u >> 6) * 64 + j], bit);
+      if (!(old & bit)) atomicAdd(&qcount[j], 1);  // a repeated key of one query sets no new bit
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int unique = 0;
+    for (int j = 0; j < nq; ++j) unique += qcount[j];
+    const bool clean = bad_s == 0 && unique == nvalid_s && total <= a.umax;
+    const bool pack = clean && static_cast<float>(total) <= a.max_union_ratio * nvalid_s;
+    a.ucount[p] = nu;
+    if (pack) {
+      a.plist[atomicAdd(a.pcount, 1)] = p;
+    } else {
+      const int b = atomicAdd(a.scount, nq);
+      for (int j = 0; j < nq; ++j) a.slist[b + j] = p * a.G + j;
+    }
+  }
+}
+
+cudaError_t launch_pack_plan(const PackArgs &a, cudaStream_t stream) {
+  const int npacks = (a.Lq + a.G - 1) / a.G;
+  const int smem = ((a.N + 31) / 32) * 8;
+  if (smem > 200 * 1024 || a.G > 64) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(pack_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  pack_plan_kernel<<<npacks, kPackThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_threshold(const SelectArgs &a, cudaStream_t stream) {
   threshold_kernel<<<a.Lb, 256, 0, stream>>>(a);
   return cudaGetLastError();

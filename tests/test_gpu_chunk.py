@@ -100,3 +100,11 @@ def test_full_size_workloads(cfg, rows, exact):
     # every query: a well-formed selection (ascending, in range, no padding since all see > topk keys)
     assert np.all(np.diff(idx, axis=1) > 0)
     assert idx.min() >= 0 and np.all(idx.max(axis=1) <= cfg.q_pos0 + np.arange(cfg.L))
+
+
+def test_small_head_chunk_uses_packing_path():
+    """H = 8 MLA heads over 2,400 queries: the attention stage packs queries per CTA."""
+    cfg = dsa_inputs.small_variant(dsa_inputs.TINY, N=8192, L=2400, topk=256, H=8)
+    inp = dsa_inputs.generate(cfg)
+    idx, out, _ = run_chunk(cfg, inp)
+    check_chunk(cfg, inp, idx, out, list(range(0, cfg.L, 61)) + [1023, 1024, cfg.L - 1])

@@ -110,3 +110,33 @@ def test_full_selection_matches_dense_causal():
     for t in (0, 1, 150, 299):
         ro, _ = oracle.dense_causal_mla(pb, t)
         assert np.linalg.norm(out[t] - ro) / np.linalg.norm(ro) <= REL_L2
+
+
+# ---- packed attention: queries with H <= 32 heads share a 64-row tile over the union of their selections
+@pytest.mark.parametrize("H,topk,L", [(8, 256, 2400), (16, 512, 1200), (32, 2048, 600)])
+def test_packed_small_head_counts(H, topk, L):
+    """Enough queries that the library packs 64 / H of them per CTA (capped to keep two waves)."""
+    N = 8192
+    q, kv = make(N, L, H, seed=H + 100)
+    idx = random_selection(N, L, topk, seed=H)
+    rows = list(range(0, L, max(1, L // 40))) + [L - 1]
+    check(q, kv, idx, 1 / math.sqrt(192), rows=rows)
+
+
+def test_packed_high_overlap_and_padding():
+    """Neighbouring queries share most keys (the case packing is for); some rows padded with -1."""
+    N, L, H, topk = 6000, 1600, 16, 256
+    q, kv = make(N, L, H, seed=21)
+    rng = np.random.default_rng(4)
+    base = np.sort(rng.choice(N - L, topk, replace=False))
+    idx = np.empty((L, topk), dtype=np.int32)
+    for t in range(L):
+        row = base.copy()
+        swap = rng.choice(topk, 16, replace=False)
+        row[swap] = rng.choice(np.arange(N - L, N - L + t + 1), 16)
+        row = np.unique(row)
+        idx[t, : len(row)] = row
+        idx[t, len(row):] = -1
+    idx[7, 100:] = -1
+    rows = list(range(0, L, 53)) + [7, L - 1]
+    check(q, kv, idx, 1 / math.sqrt(192), rows=rows)
