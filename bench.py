@@ -133,6 +133,25 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest value over all ranks (every rank must call it; identity when world == 1).
+
+    Times of a multi-GPU run are taken as the slowest rank's, so the job's
+    throughput is all ranks' work divided by that time.
+    """
+    if world <= 1:
+        return float(value)
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, steps: int, max_total_ms: float) -> float:
+    """Whole-job query tokens per second: every rank runs its own replica of the chunk."""
+    return world * tokens_per_rank * steps / (max_total_ms / 1000.0)
+
+
 def cpu_oracle_rate(cfg, inp, rows: list[int], threads: int) -> tuple[float, float]:
     """Query tokens/s of the unmodified oracle over `rows` on `threads` host threads; returns (rate, seconds)."""
     import oracle
@@ -268,12 +287,9 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
             for i, n in enumerate(stage_names):
                 stages[n] += ev[i].elapsed_time(ev[i + 1]) / args.steps
             main_launch_ms.append(ev[2].elapsed_time(ev[3]))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * cfg.L * args.steps / (total_ms / 1000.0)
+    value = job_throughput(cfg.L, world, args.steps, total_ms)
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     host = {k: v.pin_memory() for k, v in inp.items()}
@@ -300,12 +316,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * cfg.L * e2e_steps / (e2e_ms / 1000.0)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_throughput(cfg.L, world, e2e_steps, e2e_ms)
 
     # ---- roofline of the dominant kernel (main indexer pass: tensor-core contraction)
     fb = flops_and_bytes(cfg)
