@@ -10,22 +10,24 @@
 // Index -1 marks a skipped entry (llama.cpp PR #25917, discussion).
 //
 // B200 mapping.  One CTA per (query, group of 64 heads).  Per 64-key tile:
-//   * two producer warps, one per stage, gather the 64 selected rows with
-//     16-byte cp.async copies (each 8-lane group moves one 128-byte row
-//     segment, coalesced) straight into the 128-byte-swizzled UMMA operand
-//     layout; a tensor-map gather (tile::gather4) was measured to issue too
+//   * seven producer warps gather the 64 selected rows with 16-byte cp.async
+//     copies straight into the 128-byte-swizzled UMMA operand layout, two
+//     rows x 256 bytes per warp instruction, with asynchronous per-lane
+//     arrivals; a tensor-map gather (tile::gather4) was measured to issue too
 //     slowly for 1,152-byte rows;
 //   * S = Q K^T on tcgen05 (M = 64 heads, N = 64 keys, K = 576), fp32 in TMEM;
 //   * softmax warps read S from TMEM (two lanes per head row, 32 key columns
 //     each), keep a running max (rescaling the output only when the max grows
-//     by more than 2^8) and write P (bf16) to shared memory in the UMMA layout;
+//     by more than 2^8) and write P (bf16) in the UMMA layout into the rope
+//     chunk of the tile's own stage (dead once S is done), so P is
+//     double-buffered with the stages at no extra shared memory;
 //   * O += P V on tcgen05 (M = 64, N = 2 x 256 latent columns, K = 64 keys),
 //     V read in place from the gathered tile as an MN-major operand.
 // TMEM: the two 64 x 256 fp32 halves of O sit in the two half-subpartitions
 // (lanes 0-15 and 16-31 of each 32-lane quarter) of columns 0-255, the two S
-// buffers in columns 256-383.  Warp roles: warps 0 and 6 gather producers
-// (stage 0 / stage 1), warp 1 MMA issuer / TMEM owner, warps 2-5 softmax and
-// output.
+// buffers in columns 256-383.  Warp roles: warp 0 MMA issuer / TMEM owner,
+// warps 1-7 gather producers (all of them fill every tile), warps 8-11
+// softmax and output.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -43,16 +45,20 @@ constexpr int ATOMS = DIM / 64;  // 128-byte column atoms
 constexpr int ATOM_BYTES = 64 * 128;  // 64 rows x 128 B
 constexpr int Q_BYTES = ATOMS * ATOM_BYTES;
 constexpr int KV_BYTES = ATOMS * ATOM_BYTES;
-constexpr int P_BYTES = HT * BK * 2;
+constexpr int ROPE_OFF = 8 * ATOM_BYTES;  // a stage's rope chunk; holds P once S = Q K^T of its tile is done
 constexpr int STAGES = 2;
-constexpr int THREADS = 224;
+constexpr int N_PROD = 7;                            // gather producer warps
+constexpr int PPW = (BK / 2 + N_PROD - 1) / N_PROD;  // 2-row groups per producer warp
+constexpr int GPW = (BK / 4 + N_PROD - 1) / N_PROD;  // 4-row groups per producer warp
+constexpr int WARP_PROD0 = 1, WARP_SOFT0 = WARP_PROD0 + N_PROD;
+constexpr int THREADS = 32 * (WARP_SOFT0 + 4);
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + Q_BYTES;
-constexpr int OFF_P = OFF_KV + STAGES * KV_BYTES;
-constexpr int OFF_BAR = OFF_P + P_BYTES;
-constexpr int NBAR = 1 + 2 * STAGES + 4 + 2 + 1;
+constexpr int OFF_BAR = OFF_KV + STAGES * KV_BYTES;
+constexpr int NBAR = 1 + 2 * STAGES + 4 + 2 + 1 + STAGES;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int OFF_MEMB = OFF_MISC + 64;             // [STAGES][64] per-query key masks (packed mode)
+constexpr int OFF_VALID = OFF_MISC + 64;            // [STAGES][8] per-producer-warp key validity words
+constexpr int OFF_MEMB = OFF_VALID + STAGES * 8 * 8;  // [STAGES][64] per-query key masks (packed mode)
 constexpr int SMEM_BYTES = OFF_MEMB + STAGES * BK * 8 + 1024;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -72,7 +78,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *q_s = smem + OFF_Q;
   uint8_t *kv_s = smem + OFF_KV;
-  uint8_t *p_s = smem + OFF_P;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   uint64_t *q_full = bars;
   uint64_t *kv_full = bars + 1;           // [2]
@@ -80,11 +85,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t *s_full = bars + 5;            // [2]
   uint64_t *s_free = bars + 7;            // [2]
   uint64_t *p_full = bars + 9;
-  uint64_t *p_free = bars + 10;
   uint64_t *drain = bars + 11;
+  uint64_t *valid_full = bars + 12;       // [2] validity words of the stage's tile published
   unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
-  unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + OFF_MISC + 8);  // [2]
+  unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + OFF_VALID);     // [2][8]
   unsigned long long *memb_s = reinterpret_cast<unsigned long long *>(smem + OFF_MEMB);       // [2][BK]
 
   const int warp = threadIdx.x / 32;
@@ -110,24 +115,24 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_full[i], N_PROD * 32);  // one asynchronous arrival per producer lane
       mbar_init(&kv_empty[i], 1);
+      mbar_init(&valid_full[i], N_PROD);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
     }
     mbar_init(p_full, 4);
-    mbar_init(p_free, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_q);
+  if (warp == WARP_PROD0 && lane == 0) prefetch_tensormap(&tmap_q);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -136,76 +141,109 @@ __global__ void __launch_bounds__(THREADS, 1)
   const unsigned o_hi = tmem + (16u << 16);            // lanes 16-31 of each quarter, cols 0-255
   const unsigned s_col = tmem + 256;                   // S buffers: cols 256-319, 320-383
 
-  if (warp == 0 || warp == 6) {
+  if (warp >= WARP_PROD0 && warp < WARP_SOFT0) {
     // ------------------------------------------------------------ gather producers
-    // Producer p owns stage p and fills tiles p, p + 2, p + 4, ...  Lane l moves
-    // the 16-byte column chunk (l % 8) of rows 4g + l / 8 (g = 0..15) for all
-    // 9 column atoms: every 8-lane group reads one whole 128-byte segment.
-    const int p = warp == 0 ? 0 : 1;
-    const int r = lane >> 3, c8 = lane & 7;
+    // All producer warps fill every tile (tile j goes to stage j % 2).  The
+    // latent chunks go in pairs: a warp instruction moves 2 rows x 256 bytes
+    // (lane / 16 picks the row, lane / 8 % 2 the chunk of the pair, lane % 8
+    // the 16-byte piece), which gathers about twice as fast as 4 rows x 128
+    // bytes; the rope chunk goes 4 rows x 128 bytes.  Producer warp pw takes
+    // row pairs and row quads pw + N_PROD i.  Each lane's arrival on the
+    // stage's barrier fires when its copies land, so the producers never
+    // block on data and keep many rows in flight.
+    const int pw = warp - WARP_PROD0;
+    const int u = lane & 7;
+    const int sub2 = lane >> 4, seg = (lane >> 3) & 1;  // pair mapping
+    const int sub4 = lane >> 3;                         // quad mapping
     bool ok = true;
-    if (p == 0 && lane == 0) {
+    if (pw == 0 && lane == 0) {
       mbar_arrive_expect_tx(q_full, Q_BYTES);
       const int row0 = t * a.H + hg * HT;
       for (int at = 0; at < ATOMS; ++at) tma_load_2d(q_s + at * ATOM_BYTES, &tmap_q, q_full, at * 64, row0);
     }
-    auto load_idx = [&](int j, int (&v)[16]) {
+    auto key_at = [&](int j, int r) -> int {
+      const int pos = j * BK + r;
+      return (j < ntiles && pos < nkeys) ? keys[pos] : -1;
+    };
+    auto load_keys = [&](int j, int (&kp)[PPW], int (&kq)[GPW]) {
 #pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        const int pos = j * BK + 4 * g + r;
-        v[g] = (j < ntiles && pos < nkeys) ? keys[pos] : -1;
+      for (int i = 0; i < PPW; ++i) {
+        const int grp = pw + N_PROD * i;
+        kp[i] = grp < BK / 2 ? key_at(j, 2 * grp + sub2) : -1;
       }
+#pragma unroll
+      for (int i = 0; i < GPW; ++i) {
+        const int grp = pw + N_PROD * i;
+        kq[i] = grp < BK / 4 ? key_at(j, 4 * grp + sub4) : -1;
+      }
+    };
+    // Packed mode: lane q < G of producer warp 0 carries query q's 64-bit key mask of the tile.
+    auto load_mask = [&](int j) -> unsigned long long {
+      return (PACKED && pw == 0 && lane < nq && j < ntiles) ? qmask[static_cast<long long>(j) * 64 + lane] : 0ull;
+    };
+    auto row_offset = [&](int v) -> long long {  // invalid entries read row 0 (their scores are masked)
+      return static_cast<long long>((v >= 0 && v < a.N) ? v : 0) * (DIM * 2);
     };
     const uint8_t *kv = static_cast<const uint8_t *>(a.kv);
-    const unsigned stage_base = smem_u32(kv_s + p * KV_BYTES);
-    // Packed mode: lane j < G also carries query j's 64-bit key mask of the tile.
-    auto load_mask = [&](int j) -> unsigned long long {
-      return (PACKED && lane < nq && j < ntiles) ? qmask[static_cast<long long>(j) * 64 + lane] : 0ull;
-    };
-    int cur[16], nxt[16];
-    unsigned long long cur_m = 0ull, nxt_m = 0ull;
-    load_idx(p, cur);
-    cur_m = load_mask(p);
-    for (int j = p; j < ntiles; j += 2) {
-      load_idx(j + 2, nxt);
-      nxt_m = load_mask(j + 2);
-      if (!mbar_wait(&kv_empty[p], ((j >> 1) & 1) ^ 1u, abort_flag)) { ok = false; break; }
+    // Index registers run one tile ahead.
+    int kp[PPW], kq[GPW], kp_n[PPW], kq_n[GPW];
+    unsigned long long cm = 0ull, cm_n = 0ull;
+    load_keys(0, kp, kq);
+    cm = load_mask(0);
+    for (int j = 0; j < ntiles; ++j) {
+      load_keys(j + 1, kp_n, kq_n);
+      cm_n = load_mask(j + 1);
+      const int st = j & 1;
       unsigned long long vbits = 0;
-      if (PACKED && lane < nq) memb_s[p * BK + lane] = cur_m;
 #pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        const int v = cur[g];
-        const bool good = v >= 0 && v < a.N;
-        if (c8 == 0 && (v >= a.N || v < -1)) atomicOr(a.status, DEV_BAD_INDEX);
-        vbits |= static_cast<unsigned long long>(good ? 1u : 0u) << (4 * g + r);
-        const int row = good ? v : 0;
-        const int key = 4 * g + r;
-        const uint8_t *src = kv + static_cast<long long>(row) * (DIM * 2) + c8 * 16;
-        const unsigned dst = stage_base + key * 128 + ((c8 ^ (key & 7)) << 4);
-#pragma unroll
-        for (int at = 0; at < ATOMS; ++at) cp_async_16(dst + at * ATOM_BYTES, src + at * 128);
+      for (int i = 0; i < GPW; ++i) {
+        const int v = kq[i];
+        if (u == 0 && (v >= a.N || v < -1)) atomicOr(a.status, DEV_BAD_INDEX);
+        const int grp = pw + N_PROD * i;
+        if (grp < BK / 4 && v >= 0 && v < a.N) vbits |= 1ull << (4 * grp + sub4);
       }
-      cp_async_wait_all();
-      fence_proxy_async_smem();
       vbits |= __shfl_xor_sync(0xffffffffu, vbits, 8);
       vbits |= __shfl_xor_sync(0xffffffffu, vbits, 16);
+      if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1u, abort_flag)) { ok = false; break; }
+      // The stage's previous tile has been consumed (its softmax included).
+      if (PACKED && pw == 0 && lane < nq) memb_s[st * BK + lane] = cm;
       __syncwarp();
       if (lane == 0) {
-        valid_s[p] = vbits;
-        mbar_arrive(&kv_full[p]);
+        valid_s[st * 8 + pw] = vbits;
+        mbar_arrive(&valid_full[st]);
+      }
+      const unsigned stage_base = smem_u32(kv_s + st * KV_BYTES);
+#pragma unroll
+      for (int pr = 0; pr < 4; ++pr) {
+        const int c = 2 * pr + seg;
+#pragma unroll
+        for (int i = 0; i < PPW; ++i) {
+          const int r = 2 * (pw + N_PROD * i) + sub2;
+          if (r < BK)
+            cp_async_16(stage_base + c * ATOM_BYTES + r * 128 + ((u ^ (r & 7)) << 4), kv + row_offset(kp[i]) + c * 128 + u * 16);
+        }
       }
 #pragma unroll
-      for (int g = 0; g < 16; ++g) cur[g] = nxt[g];
-      cur_m = nxt_m;
+      for (int i = 0; i < GPW; ++i) {
+        const int r = 4 * (pw + N_PROD * i) + sub4;
+        if (r < BK)
+          cp_async_16(stage_base + 8 * ATOM_BYTES + r * 128 + ((u ^ (r & 7)) << 4), kv + row_offset(kq[i]) + 8 * 128 + u * 16);
+      }
+      cp_async_arrive_noinc(&kv_full[st]);
+#pragma unroll
+      for (int i = 0; i < PPW; ++i) kp[i] = kp_n[i];
+#pragma unroll
+      for (int i = 0; i < GPW; ++i) kq[i] = kq_n[i];
+      cm = cm_n;
     }
     cp_async_wait_all();  // never leave with copies in flight
     if (!ok) {
       if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
       *abort_flag = 1;
     }
-    if (p == 0 && lane == 0 && !mbar_wait(q_full, 0u, nullptr)) atomicOr(a.status, DEV_TIMEOUT);
+    if (pw == 0 && lane == 0 && !mbar_wait(q_full, 0u, nullptr)) atomicOr(a.status, DEV_TIMEOUT);
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr unsigned idesc_qk = make_idesc(HT, BK, 1u, 0u, 0u);   // S = Q K^T, both K-major
     constexpr unsigned idesc_pv = make_idesc(HT, 256, 1u, 0u, 1u);  // O += P V, V MN-major
@@ -214,21 +252,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     // address field (address >> 4; shared addresses stay below 2^18, so the
     // 14-bit field never carries).
     const uint64_t q_desc = smem_desc_sw128(smem_u32(q_s), 16, 1024);
-    const uint64_t p_desc = smem_desc_sw128(smem_u32(p_s), 16, 1024);
+    const uint64_t p_desc[2] = {smem_desc_sw128(smem_u32(kv_s + ROPE_OFF), 16, 1024),
+                                smem_desc_sw128(smem_u32(kv_s + KV_BYTES + ROPE_OFF), 16, 1024)};
     const uint64_t k_desc[2] = {smem_desc_sw128(smem_u32(kv_s), 16, 1024),
                                 smem_desc_sw128(smem_u32(kv_s + KV_BYTES), 16, 1024)};
     const uint64_t v_desc[2] = {smem_desc_sw128(smem_u32(kv_s), ATOM_BYTES, 1024),
                                 smem_desc_sw128(smem_u32(kv_s + KV_BYTES), ATOM_BYTES, 1024)};
     auto issue_pv = [&](int jj) {
       const uint64_t vd = v_desc[jj & 1];
+      const uint64_t pd = p_desc[jj & 1];
 #pragma unroll
       for (int ks = 0; ks < BK / 16; ++ks) {
         const unsigned acc = (jj > 0 || ks > 0) ? 1u : 0u;
-        mma_bf16_ss(o_lo, p_desc + ((ks * 32) >> 4), vd + ((ks * 2048) >> 4), idesc_pv, acc);
-        mma_bf16_ss(o_hi, p_desc + ((ks * 32) >> 4), vd + ((4 * ATOM_BYTES + ks * 2048) >> 4), idesc_pv, acc);
+        mma_bf16_ss(o_lo, pd + ((ks * 32) >> 4), vd + ((ks * 2048) >> 4), idesc_pv, acc);
+        mma_bf16_ss(o_hi, pd + ((ks * 32) >> 4), vd + ((4 * ATOM_BYTES + ks * 2048) >> 4), idesc_pv, acc);
       }
       tc_commit(&kv_empty[jj & 1]);
-      tc_commit(p_free);
     };
     // Event-driven issue: O += P V for tile np as soon as its P is written (it
     // frees a gather stage), otherwise S = Q K^T for tile nq once its keys have
@@ -245,6 +284,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         else if (nq < ntiles && mbar_try_wait(&kv_full[nq & 1], (nq >> 1) & 1u) &&
                  mbar_try_wait(&s_free[nq & 1], ((nq >> 1) & 1u) ^ 1u))
           action = 2;
+        // the gathered rows were written through the generic proxy
+        if (action == 2) fence_proxy_async_smem();
       }
       action = __shfl_sync(0xffffffffu, action, 0);
       if (action == 1) {
@@ -302,6 +343,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int sb = j & 1;
       if (!mbar_wait(&s_full[sb], (j >> 1) & 1u, abort_flag)) { ok = false; break; }
       tc_fence_after();
+      if (!mbar_wait(&valid_full[sb], (j >> 1) & 1u, abort_flag)) { ok = false; break; }
       uint32_t sv[32];
       tmem_ld_16x32bx2_x32(s_col + lane_base + sb * 64, sv);
       tmem_ld_wait();
@@ -314,7 +356,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int qj = row / a.H;
         vbits = qj < nq ? static_cast<unsigned>(memb_s[(j & 1) * BK + qj] >> c0) : 0u;
       } else {
-        vbits = static_cast<unsigned>(valid_s[j & 1] >> c0);
+        unsigned long long vw = 0ull;
+#pragma unroll
+        for (int w = 0; w < N_PROD; ++w) vw |= valid_s[(j & 1) * 8 + w];
+        vbits = static_cast<unsigned>(vw >> c0);
       }
       float z[32];
       float tmax = -INFINITY;
@@ -348,13 +393,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float alpha = rescale ? fast_exp2(m_old - m_used) : 1.0f;
       l = l * alpha + tsum;
       l_exact = l_exact * alpha + tsum_exact;
-      if (j > 0) {
-        if (!mbar_wait(p_free, (j - 1) & 1u, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-      }
       // Rescale O when the running max moved: lanes 0-15 own the O_lo rows and
-      // lanes 16-31 the O_hi rows of the same heads (same alpha).
+      // lanes 16-31 the O_hi rows of the same heads (same alpha).  O is idle
+      // once O += P V of the previous tile (which frees its stage) is done.
       if (__any_sync(0xffffffffu, rescale)) {
+        if (!mbar_wait(&kv_empty[(j - 1) & 1], ((j - 1) >> 1) & 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
         const unsigned obase = o_lo + lane_base;  // one 32x32b access: O_lo rows then O_hi rows
 #pragma unroll 1
         for (int ch = 0; ch < 8; ++ch) {
@@ -370,7 +414,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_st_wait();
       }
       {
-        uint8_t *prow = p_s + row * 128;
+        // P of tile j goes into the rope chunk of its own stage (dead after S = Q K^T)
+        uint8_t *prow = kv_s + (j & 1) * KV_BYTES + ROPE_OFF + row * 128;
         const int cbase = c0 >> 3;  // first 16-byte chunk of this thread's 32 columns
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -383,7 +428,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    if (ok) ok = mbar_wait(p_free, (ntiles - 1) & 1u, abort_flag);
+    if (ok) ok = mbar_wait(&kv_empty[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1u, abort_flag);
     if (!ok) {
       if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
       *abort_flag = 1;
@@ -420,7 +465,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
