@@ -10,7 +10,7 @@
 // Index -1 marks a skipped entry (llama.cpp PR #25917, discussion).
 //
 // B200 mapping.  One CTA per (query, group of 64 heads).  Per 64-key tile:
-//   * seven producer warps gather the 64 selected rows with 16-byte cp.async
+//   * eleven producer warps gather the 64 selected rows with 16-byte cp.async
 //     copies straight into the 128-byte-swizzled UMMA operand layout, two
 //     rows x 256 bytes per warp instruction, with asynchronous per-lane
 //     arrivals; a tensor-map gather (tile::gather4) was measured to issue too
@@ -26,7 +26,7 @@
 // TMEM: the two 64 x 256 fp32 halves of O sit in the two half-subpartitions
 // (lanes 0-15 and 16-31 of each 32-lane quarter) of columns 0-255, the two S
 // buffers in columns 256-383.  Warp roles: warp 0 MMA issuer / TMEM owner,
-// warps 1-7 gather producers (all of them fill every tile), warps 8-11
+// warps 1-11 gather producers (all of them fill every tile), warps 12-15
 // softmax and output.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -47,7 +47,7 @@ constexpr int Q_BYTES = ATOMS * ATOM_BYTES;
 constexpr int KV_BYTES = ATOMS * ATOM_BYTES;
 constexpr int ROPE_OFF = 8 * ATOM_BYTES;  // a stage's rope chunk; holds P once S = Q K^T of its tile is done
 constexpr int STAGES = 2;
-constexpr int N_PROD = 7;                            // gather producer warps
+constexpr int N_PROD = 11;                           // gather producer warps
 constexpr int PPW = (BK / 2 + N_PROD - 1) / N_PROD;  // 2-row groups per producer warp
 constexpr int GPW = (BK / 4 + N_PROD - 1) / N_PROD;  // 4-row groups per producer warp
 constexpr int WARP_PROD0 = 1, WARP_SOFT0 = WARP_PROD0 + N_PROD;
@@ -57,8 +57,8 @@ constexpr int OFF_KV = OFF_Q + Q_BYTES;
 constexpr int OFF_BAR = OFF_KV + STAGES * KV_BYTES;
 constexpr int NBAR = 1 + 2 * STAGES + 4 + 2 + 1 + STAGES;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int OFF_VALID = OFF_MISC + 64;            // [STAGES][8] per-producer-warp key validity words
-constexpr int OFF_MEMB = OFF_VALID + STAGES * 8 * 8;  // [STAGES][64] per-query key masks (packed mode)
+constexpr int OFF_VALID = OFF_MISC + 64;            // [STAGES][N_PROD] per-producer-warp key validity words
+constexpr int OFF_MEMB = OFF_VALID + STAGES * N_PROD * 8;  // [STAGES][64] per-query key masks (packed mode)
 constexpr int SMEM_BYTES = OFF_MEMB + STAGES * BK * 8 + 1024;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t *valid_full = bars + 12;       // [2] validity words of the stage's tile published
   unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
-  unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + OFF_VALID);     // [2][8]
+  unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + OFF_VALID);     // [2][N_PROD]
   unsigned long long *memb_s = reinterpret_cast<unsigned long long *>(smem + OFF_MEMB);       // [2][BK]
 
   const int warp = threadIdx.x / 32;
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (PACKED && pw == 0 && lane < nq) memb_s[st * BK + lane] = cm;
       __syncwarp();
       if (lane == 0) {
-        valid_s[st * 8 + pw] = vbits;
+        valid_s[st * N_PROD + pw] = vbits;
         mbar_arrive(&valid_full[st]);
       }
       const unsigned stage_base = smem_u32(kv_s + st * KV_BYTES);
@@ -230,6 +230,17 @@ __global__ void __launch_bounds__(THREADS, 1)
           cp_async_16(stage_base + 8 * ATOM_BYTES + r * 128 + ((u ^ (r & 7)) << 4), kv + row_offset(kq[i]) + 8 * 128 + u * 16);
       }
       cp_async_arrive_noinc(&kv_full[st]);
+      // Pull the next tile's rows from HBM into L2 now; its gather starts only
+      // once the other stage is consumed, about half a stage cycle from here.
+#pragma unroll
+      for (int i = 0; i < GPW; ++i) {
+        const int v = kq_n[i];
+        if (v >= 0 && v < a.N) {
+          const uint8_t *row = kv + row_offset(v);
+          prefetch_l2_line(row + u * 128);
+          if (u == 0) prefetch_l2_line(row + 8 * 128);
+        }
+      }
 #pragma unroll
       for (int i = 0; i < PPW; ++i) kp[i] = kp_n[i];
 #pragma unroll
@@ -279,10 +290,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     while (ok && np < ntiles) {
       int action = 0;
       if (lane == 0) {
-        if (np < nq && mbar_try_wait(p_full, np & 1u))
+        if (np < nq && mbar_test_wait(p_full, np & 1u))
           action = 1;
-        else if (nq < ntiles && mbar_try_wait(&kv_full[nq & 1], (nq >> 1) & 1u) &&
-                 mbar_try_wait(&s_free[nq & 1], ((nq >> 1) & 1u) ^ 1u))
+        else if (nq < ntiles && mbar_test_wait(&kv_full[nq & 1], (nq >> 1) & 1u) &&
+                 mbar_test_wait(&s_free[nq & 1], ((nq >> 1) & 1u) ^ 1u))
           action = 2;
         // the gathered rows were written through the generic proxy
         if (action == 2) fence_proxy_async_smem();
@@ -358,7 +369,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       } else {
         unsigned long long vw = 0ull;
 #pragma unroll
-        for (int w = 0; w < N_PROD; ++w) vw |= valid_s[(j & 1) * 8 + w];
+        for (int w = 0; w < N_PROD; ++w) vw |= valid_s[(j & 1) * N_PROD + w];
         vbits = static_cast<unsigned>(vw >> c0);
       }
       float z[32];

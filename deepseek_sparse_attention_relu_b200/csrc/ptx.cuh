@@ -66,6 +66,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
   return ok != 0;
 }
 
+// Non-blocking check that the phase with the given parity has completed
+// (never suspends the thread; for loops that poll several barriers).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Hint that a 128-byte global line will be read soon (into L2).
+__device__ __forceinline__ void prefetch_l2_line(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
 // Wait for the phase with the given parity to complete.  Returns false after
 // the wall-clock limit, or as soon as *abort becomes non-zero (another role of
 // the CTA gave up; pass nullptr to ignore it); the caller then unwinds.
