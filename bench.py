@@ -336,7 +336,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
-        n_rows = max(4, min(cfg.L, 6 * threads))
+        n_rows = max(4, min(cfg.L, 16 * threads))  # about 10-15 s of wall time on the 128K workload
         rows = sample_rows(cfg, n_rows)
         rate, secs = cpu_oracle_rate(cfg, inp, rows, threads)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
