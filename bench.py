@@ -344,7 +344,11 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                          f"attention), {secs:.1f} s wall on {threads} threads"}
 
     pilot_launches = 1 if cfg.q_pos0 + min(cfg.L, 1024) > 8192 else 0
-    gpu_launches = args.steps * nblocks * (5 + pilot_launches)
+    # Per query block: [pilot], threshold, main pass, select, fallback, attention; a chunk with
+    # fewer (query, 64-head group) items than half the SMs runs split-key attention plus a merge.
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    split = 2 * cfg.L * ((cfg.H + 63) // 64) <= sms and cfg.topk > 128
+    gpu_launches = args.steps * nblocks * (5 + pilot_launches + (1 if split else 0))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",

@@ -298,13 +298,43 @@ size_t union_bytes(int Lq, int topk) {
   return align256(slots * 4) + align256(slots * 8) + 3 * align256(static_cast<size_t>(Lq) * 4) + 256;
 }
 
+// Split-key attention: when a chunk has too few (query, 64-head group) items
+// to occupy the GPU (decode-like shapes), each query's selection is divided
+// among up to 16 CTAs of at least two 64-key tiles each, and the shares are
+// merged by their log-sum-exp.  Decided from the whole chunk's L, never from
+// a query block's size, so that results do not depend on the blocking.
+int mla_splits(int L, int H, int topk) {
+  const int items = L * ((H + 63) / 64);
+  const int sms = std::max(1, sm_count());
+  if (2 * items > sms) return 1;
+  return std::max(1, std::min({16, (topk + 127) / 128, sms / items}));
+}
+
+// Partial results of a block of Lq queries with ns shares each.
+size_t split_bytes(int Lq, int H, int ns) {
+  if (Lq <= 0 || ns <= 1) return 0;
+  const size_t rows = static_cast<size_t>(Lq) * H * ns;
+  return align256(rows * 512 * 4) + align256(rows * 4);
+}
+
+// Scratch of the attention stage beyond the status header: the union buffers
+// of packed attention or the partial results of split-key attention (the two
+// never occur in the same block: packing needs many queries, splitting few).
 struct UnionWorkspace {
   void *base = nullptr;
   size_t bytes = 0;
 };
 
+// Attention scratch for an L-query chunk run in blocks of QB: the larger of
+// the packing unions (H <= 32) and the split-key partials of either block size.
+size_t attention_scratch_bytes(int L, int QB, int H, int topk) {
+  const size_t b = H <= 32 ? union_bytes(QB, topk) : 0;
+  return std::max(b, split_bytes(std::min(L, QB), H, mla_splits(L, H, topk)));
+}
+
 dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, unsigned *status, int t0, int Lq,
                            cudaStream_t stream, UnionWorkspace uw = UnionWorkspace()) {
+  // p.L is the whole chunk's query count (see mla_splits).
   MlaArgs a{};
   a.topk_idx = p.topk_idx;
   a.kv = p.kv;
@@ -319,6 +349,16 @@ dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, unsigned 
   a.Lq = Lq;
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.G = 1;
+  a.nsplit = 1;
+  const int ns = mla_splits(p.L, p.H, p.topk);
+  if (ns > 1 && uw.base != nullptr && uw.bytes >= split_bytes(Lq, p.H, ns)) {
+    const size_t rows = static_cast<size_t>(Lq) * p.H * ns;
+    a.nsplit = ns;
+    a.part_o = static_cast<float *>(uw.base);
+    a.part_lse = reinterpret_cast<float *>(static_cast<uint8_t *>(uw.base) + align256(rows * 512 * 4));
+    if (!cuda_ok(launch_sparse_mla(tq, a, false, stream))) return DSA_ERR_CUDA;
+    return cuda_ok(launch_mla_combine(a, stream)) ? DSA_OK : DSA_ERR_CUDA;
+  }
   const int G = pack_group(p.H, p.topk, Lq, p.N);
   if (G >= 2 && uw.base != nullptr && uw.bytes >= union_bytes(Lq, p.topk)) {
     const int npacks = (Lq + G - 1) / G;
@@ -415,7 +455,7 @@ dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float 
 
 size_t dsa_sparse_mla_workspace(int L, int H, int topk) {
   if (L <= 0 || H <= 0 || topk <= 0) return 0;
-  return kHeaderBytes + (H <= 32 ? union_bytes(L, topk) : 0);
+  return kHeaderBytes + attention_scratch_bytes(L, L, H, topk);
 }
 
 dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, const int32_t *topk_idx, int L, int N, int H,
@@ -443,7 +483,8 @@ size_t dsa_prefill_chunk_workspace(int L, int N, int H_I, int D_I, int H, int to
   const int QB = std::min(L, query_block > 0 ? query_block : kDefaultQueryBlock);
   size_t bytes = idx_fixed_bytes(QB, N) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
   if (!want_topk_out) bytes += align256(static_cast<size_t>(QB) * topk * 4);
-  if (H <= 32) bytes += union_bytes(QB, topk) + 256;
+  const size_t extra = attention_scratch_bytes(L, QB, H, topk);
+  if (extra > 0) bytes += extra + 256;
   return bytes;
 }
 
@@ -468,16 +509,15 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, const floa
     idx_bytes = (workspace_bytes - need) & ~static_cast<size_t>(255);
     block_idx = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + idx_bytes);
   }
-  // Union buffers of the packed attention (H <= 32), below the selected keys.
+  // Attention scratch (packed-attention unions or split-key partials), below the selected keys.
   UnionWorkspace uw;
-  if (H <= 32 && workspace != nullptr) {
-    const size_t ub = union_bytes(QB, topk);
-    if (idx_bytes >= ub + (size_t(1) << 20)) {
-      const size_t off = (idx_bytes - ub) & ~static_cast<size_t>(255);
-      uw.base = static_cast<uint8_t *>(workspace) + off;
-      uw.bytes = idx_bytes - off;
-      idx_bytes = off;
-    }
+  const size_t ub = attention_scratch_bytes(L, QB, H, topk);
+  const size_t idx_need = idx_fixed_bytes(QB, N) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
+  if (ub > 0 && workspace != nullptr && idx_bytes >= ub + idx_need) {
+    const size_t off = (idx_bytes - ub) & ~static_cast<size_t>(255);
+    uw.base = static_cast<uint8_t *>(workspace) + off;
+    uw.bytes = idx_bytes - off;
+    idx_bytes = off;
   }
   IndexerProblem ip{q_idx, k_idx, w, dtype == DSA_FP8_E4M3, L, N, H_I, D_I, q_pos0, topk,
                     topk_idx_out ? topk_idx_out : block_idx, nullptr};

@@ -75,6 +75,12 @@ struct MlaArgs {
   // query in unpacked mode) and CTAs with i >= *list_count exit at once.
   const int *list;
   const int *list_count;
+  // Split-key mode (unpacked, nsplit > 1): CTA z of a query takes its z-th
+  // share of the selection and writes a partial result; a combine kernel
+  // merges the shares by their log-sum-exp.
+  int nsplit;
+  float *part_o;                  // [Lq, H, nsplit, 512] normalised partial outputs
+  float *part_lse;                // [Lq, H, nsplit] natural-log LSE of each share (-inf if empty)
 };
 
 // Union of each pack's G index rows with membership masks (packed attention).
@@ -93,5 +99,6 @@ struct PackArgs {
 cudaError_t launch_pack_plan(const PackArgs &a, cudaStream_t stream);
 
 cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, bool packed, cudaStream_t stream);
+cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t stream);
 
 }  // namespace dsa

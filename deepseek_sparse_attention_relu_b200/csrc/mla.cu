@@ -102,10 +102,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int t = a.t0 + item * (PACKED ? a.G : 1);  // first query of this CTA
   const int hg = blockIdx.y;
   const int nq = PACKED ? min(a.G, a.t0 + a.Lq - t) : 1;  // queries served
-  // Keys this CTA walks: the query's selection, or the pack's union.
-  const int nkeys = PACKED ? a.ucount[item] : a.topk;
+  // Keys this CTA walks: the query's selection (or its share of it in
+  // split-key mode), or the pack's union.
+  int nkeys = PACKED ? a.ucount[item] : a.topk;
   const int32_t *keys = PACKED ? a.ukeys + static_cast<long long>(item) * a.umax
                                : a.topk_idx + static_cast<long long>(t) * a.topk;
+  const bool split_mode = !PACKED && a.nsplit > 1;
+  const int split = blockIdx.z;
+  if (split_mode) {
+    const int per = ((nkeys + BK - 1) / BK + a.nsplit - 1) / a.nsplit * BK;  // whole tiles per share
+    const int k0 = split * per;
+    keys += k0;
+    nkeys = max(0, min(nkeys - k0, per));
+  }
   const unsigned long long *qmask = PACKED ? a.qmask + static_cast<long long>(item) * a.umax : nullptr;
   const int ntiles = max(1, (nkeys + BK - 1) / BK);
   // Output rows of the 64-row tile: global row out_row0 + r for r < row_limit.
@@ -449,12 +458,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool has_row = row < row_limit;
       const int dim0 = lane < 16 ? 0 : 256;
       uint16_t *orow = a.out + (out_row0 + row) * LAT + dim0;
+      // split-key mode: this share's normalised fp32 output row
+      const long long prow_idx = (static_cast<long long>(t - a.t0) * a.H + hg * HT + row) * a.nsplit + split;
+      float *porow = split_mode ? a.part_o + prow_idx * LAT + dim0 : nullptr;
 #pragma unroll 1
       for (int ch = 0; ch < 8; ++ch) {
         uint32_t ov[32];
         tmem_ld_32x32b_x32(o_lo + lane_base + ch * 32, ov);
         tmem_ld_wait();
-        if (has_row) {
+        if (has_row && split_mode) {
+          float4 *dst = reinterpret_cast<float4 *>(porow + ch * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
+                                 __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
+        } else if (has_row) {
           uint32_t pkd[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -467,9 +485,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
         }
       }
-      if (lane < 16 && has_row && a.lse != nullptr) {
-        a.lse[out_row0 + row] =
-            l_exact > 0.0f ? (m_used + log2f(l_exact)) * 0.69314718055994530942f : -INFINITY;
+      const float row_lse = l_exact > 0.0f ? (m_used + log2f(l_exact)) * 0.69314718055994530942f : -INFINITY;
+      if (lane < 16 && has_row && split_mode) {
+        a.part_lse[prow_idx] = row_lse;
+      } else if (lane < 16 && has_row && a.lse != nullptr) {
+        a.lse[out_row0 + row] = row_lse;
       }
     }
   }
@@ -482,13 +502,70 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+// Merge the key shares of split-key mode: one warp per (query, head) row.
+// With per-share log-sum-exps lse_s and normalised outputs o_s, the row's
+// lse = log sum_s exp(lse_s) and out = sum_s exp(lse_s - lse) o_s, which is
+// the softmax over the union of the shares (they are disjoint).
+__global__ void __launch_bounds__(256) mla_combine_kernel(MlaArgs a) {
+  const int lane = threadIdx.x % 32;
+  const long long rowg = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  if (rowg >= static_cast<long long>(a.Lq) * a.H) return;
+  const float *ls = a.part_lse + rowg * a.nsplit;
+  const float my = lane < a.nsplit ? ls[lane] : -INFINITY;
+  float m = my;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float wgt = (m == -INFINITY || my == -INFINITY) ? 0.0f : __expf(my - m);
+  float sum = wgt;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
+  // lane d16 accumulates dims [16 d16, 16 d16 + 16)
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
+  for (int sp = 0; sp < a.nsplit; ++sp) {
+    const float ws = __shfl_sync(0xffffffffu, wgt, sp) * inv;
+    if (ws == 0.0f) continue;
+    const float4 *src = reinterpret_cast<const float4 *>(a.part_o + (rowg * a.nsplit + sp) * LAT + lane * 16);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float4 v = src[e];
+      acc[4 * e] += ws * v.x;
+      acc[4 * e + 1] += ws * v.y;
+      acc[4 * e + 2] += ws * v.z;
+      acc[4 * e + 3] += ws * v.w;
+    }
+  }
+  const long long orow = (static_cast<long long>(a.t0) * a.H + rowg) * LAT + lane * 16;
+  uint32_t pk[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+    pk[e] = *reinterpret_cast<const uint32_t *>(&b);
+  }
+  uint4 *dst = reinterpret_cast<uint4 *>(a.out + orow);
+  dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  if (lane == 0 && a.lse != nullptr)
+    a.lse[static_cast<long long>(a.t0) * a.H + rowg] = sum > 0.0f ? m + logf(sum) : -INFINITY;
+}
+
 }  // namespace mla
+
+cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(a.Lq) * a.H;
+  const int blocks = static_cast<int>((rows * 32 + 255) / 256);
+  mla::mla_combine_kernel<<<blocks, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, bool packed, cudaStream_t stream) {
   auto kern = packed ? mla::sparse_mla_kernel<true> : mla::sparse_mla_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid(packed ? (a.Lq + a.G - 1) / a.G : a.Lq, packed ? 1 : (a.H + mla::HT - 1) / mla::HT);
+  dim3 grid(packed ? (a.Lq + a.G - 1) / a.G : a.Lq, packed ? 1 : (a.H + mla::HT - 1) / mla::HT,
+            packed ? 1 : max(1, a.nsplit));
   kern<<<grid, mla::THREADS, mla::SMEM_BYTES, stream>>>(tq, a);
   return cudaGetLastError();
 }

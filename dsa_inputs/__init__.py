@@ -86,7 +86,12 @@ CTX256K = ChunkConfig("dsa-256k-fp8-N262144-L8192", N=262144, L=8192, H_I=32, D_
                       seed=4)
 
 WORKLOADS = [TINY, TIES, CTX64K, CTX128K, CTX256K]
-BY_NAME = {c.name: c for c in WORKLOADS}
+# Decode: one new query over the 128K cache (the same distributions as the 128K
+# workload).  Not one of the five benchmark workloads; a latency case.
+DECODE128K = ChunkConfig("dsa-decode-128k-N131072-L1", N=131072, L=1, H_I=32, D_I=128, idx_dtype="bf16",
+                         idx_dist="normal", w_dist="normal_rsqrt", topk=2048, H=64, lat_std=0.5, rope_std=0.5,
+                         seed=3)
+BY_NAME = {c.name: c for c in WORKLOADS + [DECODE128K]}
 
 
 def small_variant(cfg: ChunkConfig, N: int, L: int, topk: int | None = None, H: int | None = None,

@@ -108,3 +108,12 @@ def test_small_head_chunk_uses_packing_path():
     inp = dsa_inputs.generate(cfg)
     idx, out, _ = run_chunk(cfg, inp)
     check_chunk(cfg, inp, idx, out, list(range(0, cfg.L, 61)) + [1023, 1024, cfg.L - 1])
+
+
+def test_decode_chunk_split_key():
+    """One query over the 128K cache (decode): the attention stage runs split-key."""
+    cfg = dsa_inputs.small_variant(dsa_inputs.CTX128K, N=131072, L=1, topk=2048, H=64)
+    inp = dsa_inputs.generate(cfg)
+    idx, out, lse = run_chunk(cfg, inp)
+    assert np.isfinite(lse.cpu().numpy()).all()
+    check_chunk(cfg, inp, idx, out, [0])

@@ -140,3 +140,24 @@ def test_packed_high_overlap_and_padding():
     idx[7, 100:] = -1
     rows = list(range(0, L, 53)) + [7, L - 1]
     check(q, kv, idx, 1 / math.sqrt(192), rows=rows)
+
+
+# ---- split-key attention: blocks with too few queries to fill the GPU (decode) divide each
+# ---- query's selection among several CTAs and merge the shares by their log-sum-exp
+@pytest.mark.parametrize("N,L,H,topk,pad", [(131072, 1, 64, 2048, 0), (131072, 1, 128, 2048, 0),
+                                            (5000, 3, 64, 300, 0), (9000, 2, 64, 1000, 400)])
+def test_decode_split_key(N, L, H, topk, pad):
+    q, kv = make(N, L, H, seed=N % 97 + H)
+    idx = random_selection(N, L, topk, seed=L + H, pad=pad)
+    check(q, kv, idx, 1 / math.sqrt(192))
+
+
+def test_decode_split_key_empty_shares():
+    """Shares left with no valid key (all -1) contribute nothing; an all-padding row is zero with LSE -inf."""
+    N, L, H, topk = 4000, 2, 64, 1024
+    q, kv = make(N, L, H, seed=31)
+    idx = np.full((L, topk), -1, dtype=np.int32)
+    idx[0, :100] = np.sort(np.random.default_rng(2).choice(N, 100, replace=False))  # only the first share has keys
+    out, lse = run_mla(q, kv, idx, 1 / math.sqrt(192))
+    assert np.all(out[1] == 0.0) and np.all(np.isneginf(lse[1]))
+    check(q, kv, idx, 1 / math.sqrt(192), rows=[0])
