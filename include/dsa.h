@@ -126,7 +126,12 @@ dsa_status_t dsa_indexer_topk_noalloc(const void *q_idx, const void *k_idx, cons
                                       int L, int N, int H_I, int D_I, int q_pos0, int topk, int32_t *topk_idx,
                                       float *topk_score, dsa_stream_t stream);
 
-/* Workspace (bytes) for dsa_sparse_mla_prefill: the status word only. */
+/* Workspace (bytes) for dsa_sparse_mla_prefill: the status word, plus the
+ * union buffers of packed attention (H <= 32) or the fp32 partial results of
+ * split-key attention (chunks with few queries), whichever is larger; the
+ * size depends on the current device's SM count.  A smaller workspace (at
+ * least the status word) is accepted: the call then runs neither packed nor
+ * split, with the same results up to rounding. */
 size_t dsa_sparse_mla_workspace(int L, int H, int topk);
 
 /*
@@ -144,6 +149,15 @@ size_t dsa_sparse_mla_workspace(int L, int H, int topk);
  *   out = sum_j softmax(z)_j * kv_lat[i_j]    (fp32 accumulate, bf16 out)
  *
  * Supported: any H >= 1 (processed in groups of 64 heads), topk >= 1.
+ *
+ * Scheduling (results are the same up to fp32 rounding order):
+ *   - H <= 32 and many queries: neighbouring queries whose selections share
+ *     most keys are packed into one CTA over the union of their keys;
+ *   - L * ceil(H / 64) below half the SM count (decode-like chunks): each
+ *     query's selection is split into up to 16 shares of at least 128 keys,
+ *     attended by separate CTAs and merged by their log-sum-exp (a second
+ *     kernel).  The choice depends on L, H and topk only, never on a caller's
+ *     query blocking.
  */
 dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, const int32_t *topk_idx, int L, int N, int H,
                                     int topk, float scale, void *out, float *lse, void *workspace,
