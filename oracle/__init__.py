@@ -58,14 +58,16 @@ def lib() -> ctypes.CDLL:
         L.oracle_e4m3_value.restype = d
         L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
         L.oracle_indexer_scores.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P]
+        L.oracle_indexer_scores_range.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, P]
         L.oracle_topk_fullsort.argtypes = [P, i32, i32, P, P]
         L.oracle_topk_blocked_fold.argtypes = [P, i32, i32, i32, P]
         L.oracle_sparse_mla.argtypes = [P, P, P, i32, i32, i32, i32, d, i32, P, P]
         L.oracle_dense_causal_mla.argtypes = [P, P, i32, i32, i32, i32, d, i32, P, P]
         L.oracle_prefill_row.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, i32, d, i32,
                                          P, P, P, P]
-        for name in ("oracle_indexer_scores", "oracle_topk_fullsort", "oracle_topk_blocked_fold",
-                     "oracle_sparse_mla", "oracle_dense_causal_mla", "oracle_prefill_row", "oracle_version"):
+        for name in ("oracle_indexer_scores", "oracle_indexer_scores_range", "oracle_topk_fullsort",
+                     "oracle_topk_blocked_fold", "oracle_sparse_mla", "oracle_dense_causal_mla", "oracle_prefill_row",
+                     "oracle_version"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -108,6 +110,22 @@ def indexer_scores(pb: Problem, t: int) -> np.ndarray:
     _check(lib().oracle_indexer_scores(_ptr(pb.q_idx), _ptr(pb.k_idx), _ptr(pb.w), pb.idx_dtype, pb.L, pb.N,
                                        pb.H_I, pb.D_I, pb.q_pos0, t, _ptr(out)), "indexer_scores")
     return out
+
+
+def indexer_scores_range(pb: Problem, t: int, lo: int, hi: int) -> np.ndarray:
+    """Scores of query t over keys [lo, hi) (general causality through an index mask)."""
+    out = np.empty(max(0, hi - lo), dtype=np.float64)
+    _check(lib().oracle_indexer_scores_range(_ptr(pb.q_idx), _ptr(pb.k_idx), _ptr(pb.w), pb.idx_dtype, pb.L,
+                                             pb.N, pb.H_I, pb.D_I, lo, hi, t, _ptr(out)), "indexer_scores_range")
+    return out
+
+
+def topk_row_range(pb: Problem, t: int, lo: int, hi: int):
+    """(selected keys ascending with -1 padding, k-th score, score row of [lo, hi)) of query t over its range."""
+    s = indexer_scores_range(pb, t, lo, hi)
+    idx, kth = topk_fullsort(s, pb.topk)
+    idx = np.where(idx >= 0, idx + lo, -1).astype(np.int32)
+    return idx, kth, s
 
 
 def topk_fullsort(scores: np.ndarray, topk: int):

@@ -26,7 +26,8 @@
  *     ReLU per head before the signed head weight, one indexer key per position
  *     shared by all indexer heads;
  *   - causality is inclusive: query t sits at position p_t = q_pos0 + t and sees
- *     keys s <= p_t;
+ *     keys s <= p_t; with general causality (an index mask) query t sees the
+ *     keys of its own half-open range [lo_t, hi_t);
  *   - ties in I are broken toward the smaller key index;
  *   - the selected set is emitted in ascending key order, then -1 padding when
  *     fewer than topk keys are visible;
@@ -113,6 +114,41 @@ int oracle_indexer_scores(const void *q_idx, const void *k_idx, const float *w, 
             score += (double)w[(int64_t)t * H_I + h] * relu;
         }
         out[s] = score;
+    }
+    free(q);
+    free(k);
+    return ORACLE_OK;
+}
+
+/*
+ * Lightning-indexer scores of query row t over the keys of a half-open range
+ * [lo, hi): general causality carried by the index mask, [LCPP] discussion
+ * (causality applied to the indices rather than assumed triangular, so that
+ * a unified cache holding several sequences, or a non-triangular mask, is
+ * expressed per query).  The same formula and loop order as
+ * oracle_indexer_scores; out receives hi - lo doubles, out[j] for key lo + j.
+ * Requires 0 <= lo <= hi <= N; positions play no further role.
+ */
+int oracle_indexer_scores_range(const void *q_idx, const void *k_idx, const float *w, int dtype,
+                                int L, int N, int H_I, int D_I, int lo, int hi, int t, double *out) {
+    if (t < 0 || t >= L || lo < 0 || hi < lo || hi > N || H_I <= 0 || D_I <= 0) return ORACLE_EINVAL;
+    if (dtype != ORACLE_IDX_BF16 && dtype != ORACLE_IDX_E4M3) return ORACLE_EINVAL;
+    double *q = (double *)malloc(sizeof(double) * (size_t)H_I * D_I);
+    double *k = (double *)malloc(sizeof(double) * (size_t)D_I);
+    if (!q || !k) { free(q); free(k); return ORACLE_ENOMEM; }
+    for (int h = 0; h < H_I; ++h)
+        for (int d = 0; d < D_I; ++d)
+            q[h * D_I + d] = idx_value(q_idx, dtype, ((int64_t)t * H_I + h) * D_I + d);
+    for (int s = lo; s < hi; ++s) {
+        for (int d = 0; d < D_I; ++d) k[d] = idx_value(k_idx, dtype, (int64_t)s * D_I + d);
+        double score = 0.0;
+        for (int h = 0; h < H_I; ++h) {
+            double dot = 0.0;
+            for (int d = 0; d < D_I; ++d) dot += q[h * D_I + d] * k[d];
+            double relu = dot > 0.0 ? dot : 0.0;
+            score += (double)w[(int64_t)t * H_I + h] * relu;
+        }
+        out[s - lo] = score;
     }
     free(q);
     free(k);

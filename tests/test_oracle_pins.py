@@ -150,6 +150,40 @@ def test_integer_inputs_scores_exact(oracle_lib):
         assert np.array_equal(oracle.indexer_scores(pb, t), want)
 
 
+def test_range_scores_integer_exact(oracle_lib):
+    """Per-query key ranges (general causality): on integer inputs the scores of keys [lo, hi) equal an
+    int64 matmul over exactly those key rows, whatever the query's position (a shifted or clipped range
+    fails)."""
+    cfg = dsa_inputs.small_variant(dsa_inputs.TIES, N=2048, L=8, topk=256)
+    inp = dsa_inputs.generate(cfg, with_mla=False)
+    pb = oracle_problem(cfg, inp)
+    k = inp["k_idx"].to(torch.int64)
+    for t, lo, hi in [(0, 0, 2048), (3, 100, 101), (5, 1500, 2048), (7, 700, 1300), (2, 40, 40)]:
+        q = inp["q_idx"][t].to(torch.int64)
+        dots = torch.clamp(k[lo:hi] @ q.T, min=0)
+        want = (dots * inp["w"][t].to(torch.int64)).sum(1).numpy().astype(np.float64)
+        got = oracle.indexer_scores_range(pb, t, lo, hi)
+        assert got.shape == (hi - lo,) and np.array_equal(got, want)
+    # the causal row is the range [0, q_pos0 + t + 1)
+    assert np.array_equal(oracle.indexer_scores_range(pb, 4, 0, cfg.q_pos0 + 5), oracle.indexer_scores(pb, 4))
+
+
+def test_range_topk_is_lexsort_of_the_slice(oracle_lib):
+    """Top-k over a range = the (score desc, key asc) sort of that slice, reported as absolute keys;
+    -1 padding when the range holds fewer than k keys; an empty range selects nothing."""
+    cfg = dsa_inputs.small_variant(dsa_inputs.TIES, N=2048, L=4, topk=64)
+    inp = dsa_inputs.generate(cfg, with_mla=False)
+    pb = oracle_problem(cfg, inp)
+    for t, lo, hi in [(0, 300, 1800), (1, 1000, 1040), (2, 7, 7), (3, 0, 2048)]:
+        idx, kth, s = oracle.topk_row_range(pb, t, lo, hi)
+        want = _lexsort_topk(s, cfg.topk)
+        want = np.where(want >= 0, want + lo, -1)
+        assert np.array_equal(idx, want)
+        assert np.all((idx == -1) | ((idx >= lo) & (idx < hi)))
+        if hi - lo <= cfg.topk:
+            assert kth == -math.inf and np.count_nonzero(idx >= 0) == hi - lo
+
+
 # ---------------------------------------------------------------- top-k
 
 def _lexsort_topk(scores, k):
