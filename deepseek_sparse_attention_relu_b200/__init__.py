@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 EXPORTED = ("dsa_version", "dsa_status_string", "dsa_last_error_string", "dsa_indexer_topk_workspace", "dsa_indexer_topk",
             "dsa_sparse_mla_workspace", "dsa_sparse_mla_prefill", "dsa_prefill_chunk_workspace",
             "dsa_prefill_chunk", "dsa_prefill_chunk_profiled", "dsa_workspace_status",
-            "dsa_indexer_topk_noalloc")
+            "dsa_indexer_topk_noalloc", "dsa_indexer_topk_ranges", "dsa_prefill_chunk_ranges")
 
 _lib = None
 
@@ -72,6 +72,10 @@ def lib() -> ctypes.CDLL:
         L.dsa_prefill_chunk_profiled.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, I, P, P, P, P, Z, P, P, I]
         L.dsa_indexer_topk_noalloc.restype = I
         L.dsa_indexer_topk_noalloc.argtypes = [P, P, P, I, I, I, I, I, I, I, P, P, P]
+        L.dsa_indexer_topk_ranges.restype = I
+        L.dsa_indexer_topk_ranges.argtypes = [P, P, P, I, I, I, I, I, P, P, I, P, P, P, Z, P]
+        L.dsa_prefill_chunk_ranges.restype = I
+        L.dsa_prefill_chunk_ranges.argtypes = [P, P, P, I, P, P, I, I, I, I, I, P, P, I, F, I, P, P, P, P, Z, P]
         L.dsa_workspace_status.restype = I
         L.dsa_workspace_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint)]
         _lib = L
@@ -152,6 +156,29 @@ def dsa_indexer_topk(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, 
         "dsa_indexer_topk")
 
 
+def dsa_indexer_topk_ranges(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, key_lo: torch.Tensor,
+                            key_hi: torch.Tensor, topk: int, topk_idx: torch.Tensor,
+                            topk_score: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                            stream=None) -> None:
+    """dsa_indexer_topk with general visibility: query t sees keys key_lo[t] <= s < key_hi[t] (int32 CUDA
+    tensors [L]) instead of the causal prefix."""
+    L, H_I, D_I = q_idx.shape
+    N = k_idx.shape[0]
+    dt = _dtype_code(q_idx)
+    if k_idx.dtype != q_idx.dtype or k_idx.shape[1] != D_I or tuple(w.shape) != (L, H_I):
+        raise ValueError("inconsistent indexer operand shapes or dtypes")
+    if tuple(topk_idx.shape) != (L, topk) or key_lo.numel() != L or key_hi.numel() != L:
+        raise ValueError("topk_idx must be [L, topk] and key_lo / key_hi [L]")
+    if workspace is None:
+        workspace = alloc_workspace(dsa_indexer_topk_workspace(L, N, H_I, D_I, topk, dt), q_idx.device)
+    _check(lib().dsa_indexer_topk_ranges(
+        _dev(q_idx, "q_idx"), _dev(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt, L, N, H_I, D_I,
+        _dev(key_lo, "key_lo", (torch.int32,)), _dev(key_hi, "key_hi", (torch.int32,)), topk,
+        _dev(topk_idx, "topk_idx", (torch.int32,)), _dev(topk_score, "topk_score", (torch.float32,)),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)),
+        "dsa_indexer_topk_ranges")
+
+
 def dsa_indexer_topk_noalloc(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, q_pos0: int, topk: int,
                              topk_idx: torch.Tensor, topk_score: torch.Tensor | None = None, stream=None) -> None:
     """dsa_indexer_topk without a workspace, for callers that cannot allocate device memory (inside CUDA graph
@@ -209,6 +236,29 @@ def dsa_prefill_chunk(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor,
         float(scale), query_block, _dev(topk_idx, "topk_idx", (torch.int32,)), _dev(out, "out", (torch.bfloat16,)),
         _dev(lse, "lse", (torch.float32,)), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)), "dsa_prefill_chunk")
+
+
+def dsa_prefill_chunk_ranges(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, q: torch.Tensor,
+                             kv: torch.Tensor, key_lo: torch.Tensor, key_hi: torch.Tensor, topk: int, scale: float,
+                             out: torch.Tensor, topk_idx: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                             query_block: int = 0, workspace: torch.Tensor | None = None, stream=None) -> None:
+    """dsa_prefill_chunk with general visibility: query t sees keys key_lo[t] <= s < key_hi[t]."""
+    L, H_I, D_I = q_idx.shape
+    N = k_idx.shape[0]
+    H = q.shape[1]
+    dt = _dtype_code(q_idx)
+    if key_lo.numel() != L or key_hi.numel() != L:
+        raise ValueError("key_lo / key_hi must have one entry per query")
+    if workspace is None:
+        workspace = alloc_workspace(dsa_prefill_chunk_workspace(L, N, H_I, D_I, H, topk, query_block, dt,
+                                                                topk_idx is not None), q.device)
+    _check(lib().dsa_prefill_chunk_ranges(
+        _dev(q_idx, "q_idx"), _dev(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt,
+        _dev(q, "q", (torch.bfloat16,)), _dev(kv, "kv", (torch.bfloat16,)), L, N, H_I, D_I, H,
+        _dev(key_lo, "key_lo", (torch.int32,)), _dev(key_hi, "key_hi", (torch.int32,)), topk, float(scale),
+        query_block, _dev(topk_idx, "topk_idx", (torch.int32,)), _dev(out, "out", (torch.bfloat16,)),
+        _dev(lse, "lse", (torch.float32,)), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "dsa_prefill_chunk_ranges")
 
 
 def dsa_prefill_chunk_profiled(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, q: torch.Tensor,

@@ -35,6 +35,7 @@ bool cuda_ok(cudaError_t e) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -81,7 +82,7 @@ int default_cap(int topk) { return std::max(kMinCap, 4 * topk); }
 
 // Fixed part of the indexer workspace (everything but the candidate lists).
 size_t idx_fixed_bytes(int QB, int N) {
-  return kHeaderBytes + 3 * align256(static_cast<size_t>(QB) * 4) +
+  return kHeaderBytes + 5 * align256(static_cast<size_t>(QB) * 4) + 2 * align256((QB + 2) * sizeof(int)) +
          align256(static_cast<size_t>(QB) * kSamples * 4) + align256(static_cast<size_t>(kFallbackSlots) * N * 4);
 }
 
@@ -94,6 +95,8 @@ struct IdxWorkspace {
   float *dense;
   float *fb_scratch;
   unsigned long long *cand;
+  int *rlo, *rhi;                 // [QB] clamped per-query key ranges (ranges mode)
+  int *grp_tile0, *grp_start;     // per-group tile windows (ranges mode)
   int cap;
 };
 
@@ -110,6 +113,14 @@ bool carve_idx_ws(void *ws, size_t bytes, int QB, int N, IdxWorkspace *o) {
   p += align256(static_cast<size_t>(QB) * 4);
   o->fb_list = reinterpret_cast<int *>(p);
   p += align256(static_cast<size_t>(QB) * 4);
+  o->rlo = reinterpret_cast<int *>(p);
+  p += align256(static_cast<size_t>(QB) * 4);
+  o->rhi = reinterpret_cast<int *>(p);
+  p += align256(static_cast<size_t>(QB) * 4);
+  o->grp_tile0 = reinterpret_cast<int *>(p);
+  p += align256((QB + 2) * sizeof(int));
+  o->grp_start = reinterpret_cast<int *>(p);
+  p += align256((QB + 2) * sizeof(int));
   o->dense = reinterpret_cast<float *>(p);
   p += align256(static_cast<size_t>(QB) * kSamples * 4);
   o->fb_scratch = reinterpret_cast<float *>(p);
@@ -127,6 +138,8 @@ struct IndexerProblem {
   int L, N, H_I, D_I, q_pos0, topk;
   int32_t *topk_idx;
   float *topk_score;
+  // Per-query key ranges (device, [L]; nullptr = causal from q_pos0).
+  const int32_t *key_lo = nullptr, *key_hi = nullptr;
 };
 
 dsa_status_t check_indexer_args(const IndexerProblem &p) {
@@ -135,8 +148,13 @@ dsa_status_t check_indexer_args(const IndexerProblem &p) {
   if (!aligned16(p.q_idx) || !aligned16(p.k_idx) || !aligned16(p.w) || !aligned16(p.topk_idx))
     return DSA_ERR_INVALID_ARG;
   if (p.topk_score != nullptr && !aligned16(p.topk_score)) return DSA_ERR_INVALID_ARG;
-  if (p.L <= 0 || p.N <= 0 || p.H_I <= 0 || p.D_I <= 0 || p.topk <= 0 || p.q_pos0 < 0) return DSA_ERR_INVALID_ARG;
-  if (static_cast<long long>(p.q_pos0) + p.L > p.N) return DSA_ERR_INVALID_ARG;
+  if (p.L <= 0 || p.N <= 0 || p.H_I <= 0 || p.D_I <= 0 || p.topk <= 0) return DSA_ERR_INVALID_ARG;
+  if ((p.key_lo == nullptr) != (p.key_hi == nullptr)) return DSA_ERR_INVALID_ARG;
+  if (p.key_lo == nullptr) {
+    if (p.q_pos0 < 0 || static_cast<long long>(p.q_pos0) + p.L > p.N) return DSA_ERR_INVALID_ARG;
+  } else if (!aligned4(p.key_lo) || !aligned4(p.key_hi)) {
+    return DSA_ERR_INVALID_ARG;
+  }
   if (p.topk > kMaxTopk) return DSA_ERR_UNSUPPORTED;
   if (!indexer_supported(p.D_I, p.H_I, p.fp8)) return DSA_ERR_UNSUPPORTED;
   return DSA_OK;
@@ -172,12 +190,37 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
   ia.q_pos0 = q_pos0;
   ia.q_row0 = t0 * p.H_I;
 
-  const bool pilot = static_cast<long long>(q_pos0) + Lb > ws.cap;
-  int n_samples = 0;
+  const bool ranges = p.key_lo != nullptr;
   if (!mark(ev, 0, stream)) return DSA_ERR_CUDA;
+  if (ranges) {
+    // Clamp the block's ranges and plan the indexer's per-group key windows.
+    RangePlanArgs ra{};
+    ra.lo_in = p.key_lo + t0;
+    ra.hi_in = p.key_hi + t0;
+    ra.lo = ws.rlo;
+    ra.hi = ws.rhi;
+    ra.grp_tile0 = ws.grp_tile0;
+    ra.grp_start = ws.grp_start;
+    ra.status = ws.status;
+    ra.Lb = Lb;
+    ra.QG = QG;
+    ra.N = p.N;
+    if (!cuda_ok(launch_range_plan(ra, stream))) return DSA_ERR_CUDA;
+    ia.key_lo = ws.rlo;
+    ia.key_hi = ws.rhi;
+    ia.grp_tile0 = ws.grp_tile0;
+    ia.grp_start = ws.grp_start;
+  }
+  // The pilot samples the keys a query can see: with ranges (unknown on the
+  // host) it samples the whole cache and each query uses the samples inside
+  // its own range.
+  const long long sampled = ranges ? p.N : static_cast<long long>(q_pos0) + 1;
+  const bool pilot = ranges ? p.N > ws.cap : static_cast<long long>(q_pos0) + Lb > ws.cap;
+  int n_samples = 0;
+  long long stride = 1;
   if (pilot) {
-    n_samples = std::min(kSamples, q_pos0 + 1);
-    const long long stride = (static_cast<long long>(q_pos0) + 1) / n_samples;
+    n_samples = static_cast<int>(std::min<long long>(kSamples, sampled));
+    stride = sampled / n_samples;
     CUtensorMap ts;
     const CUtensorMapDataType dt = p.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!make_map_2d(&ts, p.k_idx, dt, p.D_I, n_samples, stride * row_bytes, 128 / esz, 128)) return DSA_ERR_CUDA;
@@ -211,6 +254,9 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
   sa.t0 = t0;
   sa.Lb = Lb;
   sa.q_pos0 = q_pos0;
+  sa.key_lo = ranges ? ws.rlo : nullptr;
+  sa.key_hi = ranges ? ws.rhi : nullptr;
+  sa.sample_stride = static_cast<int>(stride);
   sa.N = p.N;
   sa.H_I = p.H_I;
   sa.D_I = p.D_I;
@@ -224,10 +270,14 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
   ea.pilot = 0;
   ea.n_keys = p.N;
   long long total = 0;
-  for (int g = 0; g < G; ++g) {
-    const int last = std::min(Lb, (g + 1) * QG);
-    const long long keys = std::min<long long>(p.N, static_cast<long long>(q_pos0) + last);
-    total += (keys + 127) / 128;
+  if (ranges) {
+    total = static_cast<long long>(G) * ((p.N + 127) / 128);  // an upper bound; the kernel reads the plan
+  } else {
+    for (int g = 0; g < G; ++g) {
+      const int last = std::min(Lb, (g + 1) * QG);
+      const long long keys = std::min<long long>(p.N, static_cast<long long>(q_pos0) + last);
+      total += (keys + 127) / 128;
+    }
   }
   if (total > (1ll << 30)) return DSA_ERR_UNSUPPORTED;
   ea.total_tiles = static_cast<int>(total);
@@ -432,11 +482,18 @@ size_t dsa_indexer_topk_workspace(int L, int N, int H_I, int D_I, int topk, dsa_
   return idx_fixed_bytes(QB, N) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
 }
 
-dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype, int L,
-                              int N, int H_I, int D_I, int q_pos0, int topk, int32_t *topk_idx, float *topk_score,
-                              void *workspace, size_t workspace_bytes, dsa_stream_t stream_) {
+}  // extern "C"
+
+namespace {
+
+dsa_status_t indexer_topk_impl(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype, int L,
+                               int N, int H_I, int D_I, int q_pos0, const int32_t *key_lo, const int32_t *key_hi,
+                               int topk, int32_t *topk_idx, float *topk_score, void *workspace,
+                               size_t workspace_bytes, dsa_stream_t stream_) {
   if (dtype != DSA_BF16 && dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID_ARG;
   IndexerProblem p{q_idx, k_idx, w, dtype == DSA_FP8_E4M3, L, N, H_I, D_I, q_pos0, topk, topk_idx, topk_score};
+  p.key_lo = key_lo;
+  p.key_hi = key_hi;
   dsa_status_t st = check_indexer_args(p);
   if (st != DSA_OK) return st;
   const int QB = std::min(L, kDefaultQueryBlock);
@@ -451,6 +508,26 @@ dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float 
     if (st != DSA_OK) return st;
   }
   return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype, int L,
+                              int N, int H_I, int D_I, int q_pos0, int topk, int32_t *topk_idx, float *topk_score,
+                              void *workspace, size_t workspace_bytes, dsa_stream_t stream) {
+  return indexer_topk_impl(q_idx, k_idx, w, dtype, L, N, H_I, D_I, q_pos0, nullptr, nullptr, topk, topk_idx,
+                           topk_score, workspace, workspace_bytes, stream);
+}
+
+dsa_status_t dsa_indexer_topk_ranges(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
+                                     int L, int N, int H_I, int D_I, const int32_t *key_lo,
+                                     const int32_t *key_hi, int topk, int32_t *topk_idx, float *topk_score,
+                                     void *workspace, size_t workspace_bytes, dsa_stream_t stream) {
+  if (key_lo == nullptr || key_hi == nullptr) return DSA_ERR_INVALID_ARG;
+  return indexer_topk_impl(q_idx, k_idx, w, dtype, L, N, H_I, D_I, 0, key_lo, key_hi, topk, topk_idx, topk_score,
+                           workspace, workspace_bytes, stream);
 }
 
 size_t dsa_sparse_mla_workspace(int L, int H, int topk) {
@@ -494,9 +571,9 @@ namespace {
 
 dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
                                 const void *q, const void *kv, int L, int N, int H_I, int D_I, int H, int q_pos0,
-                                int topk, float scale, int query_block, int32_t *topk_idx_out, void *out, float *lse,
-                                void *workspace, size_t workspace_bytes, dsa_stream_t stream_, cudaEvent_t *events,
-                                int n_events) {
+                                const int32_t *key_lo, const int32_t *key_hi, int topk, float scale,
+                                int query_block, int32_t *topk_idx_out, void *out, float *lse, void *workspace,
+                                size_t workspace_bytes, dsa_stream_t stream_, cudaEvent_t *events, int n_events) {
   if (dtype != DSA_BF16 && dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID_ARG;
   if (L <= 0 || topk <= 0) return DSA_ERR_INVALID_ARG;
   const int QB = std::min(L, query_block > 0 ? query_block : kDefaultQueryBlock);
@@ -521,6 +598,8 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, const floa
   }
   IndexerProblem ip{q_idx, k_idx, w, dtype == DSA_FP8_E4M3, L, N, H_I, D_I, q_pos0, topk,
                     topk_idx_out ? topk_idx_out : block_idx, nullptr};
+  ip.key_lo = key_lo;
+  ip.key_hi = key_hi;
   dsa_status_t st = check_indexer_args(ip);
   if (st != DSA_OK) return st;
   MlaProblem mp{q, kv, ip.topk_idx, L, N, H, topk, scale, out, lse};
@@ -561,8 +640,18 @@ dsa_status_t dsa_prefill_chunk(const void *q_idx, const void *k_idx, const float
                                const void *q, const void *kv, int L, int N, int H_I, int D_I, int H, int q_pos0,
                                int topk, float scale, int query_block, int32_t *topk_idx_out, void *out, float *lse,
                                void *workspace, size_t workspace_bytes, dsa_stream_t stream) {
-  return prefill_chunk_impl(q_idx, k_idx, w, dtype, q, kv, L, N, H_I, D_I, H, q_pos0, topk, scale, query_block,
-                            topk_idx_out, out, lse, workspace, workspace_bytes, stream, nullptr, 0);
+  return prefill_chunk_impl(q_idx, k_idx, w, dtype, q, kv, L, N, H_I, D_I, H, q_pos0, nullptr, nullptr, topk, scale,
+                            query_block, topk_idx_out, out, lse, workspace, workspace_bytes, stream, nullptr, 0);
+}
+
+dsa_status_t dsa_prefill_chunk_ranges(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
+                                      const void *q, const void *kv, int L, int N, int H_I, int D_I, int H,
+                                      const int32_t *key_lo, const int32_t *key_hi, int topk, float scale,
+                                      int query_block, int32_t *topk_idx_out, void *out, float *lse,
+                                      void *workspace, size_t workspace_bytes, dsa_stream_t stream) {
+  if (key_lo == nullptr || key_hi == nullptr) return DSA_ERR_INVALID_ARG;
+  return prefill_chunk_impl(q_idx, k_idx, w, dtype, q, kv, L, N, H_I, D_I, H, 0, key_lo, key_hi, topk, scale,
+                            query_block, topk_idx_out, out, lse, workspace, workspace_bytes, stream, nullptr, 0);
 }
 
 dsa_status_t dsa_prefill_chunk_profiled(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
@@ -571,8 +660,8 @@ dsa_status_t dsa_prefill_chunk_profiled(const void *q_idx, const void *k_idx, co
                                         void *out, float *lse, void *workspace, size_t workspace_bytes,
                                         dsa_stream_t stream, void *const *events, int n_events) {
   if (events == nullptr) return DSA_ERR_INVALID_ARG;
-  return prefill_chunk_impl(q_idx, k_idx, w, dtype, q, kv, L, N, H_I, D_I, H, q_pos0, topk, scale, query_block,
-                            topk_idx_out, out, lse, workspace, workspace_bytes, stream,
+  return prefill_chunk_impl(q_idx, k_idx, w, dtype, q, kv, L, N, H_I, D_I, H, q_pos0, nullptr, nullptr, topk, scale,
+                            query_block, topk_idx_out, out, lse, workspace, workspace_bytes, stream,
                             reinterpret_cast<cudaEvent_t *>(const_cast<void **>(events)), n_events);
 }
 

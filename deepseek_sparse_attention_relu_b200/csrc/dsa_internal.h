@@ -24,7 +24,26 @@ struct IndexerArgs {
   int q_row0;                     // first row of the block in the [L*H_I, D_I] query tensor map
   int total_tiles;                // sum over query groups of their 128-key tiles
   int pilot;                      // 1 = PILOT mode
+  // Per-query key ranges (general causality; nullptr = causal, query tl sees
+  // keys <= q_pos0 + tl): query tl of the block sees keys key_lo[tl] <=
+  // s < key_hi[tl].  Then group g covers the 128-key tiles grp_tile0[g] ..
+  // grp_tile0[g] + grp_start[g+1] - grp_start[g] - 1, and grp_start[G] is
+  // the total (total_tiles is ignored).
+  const int *key_lo, *key_hi;     // [Lb] clamped ranges
+  const int *grp_tile0;           // [G]
+  const int *grp_start;           // [G + 1] exclusive prefix of the groups' tile counts
 };
+
+// Clamp the block's ranges into [0, N] (flagging bad ones) and plan the
+// indexer's per-group tile windows.
+struct RangePlanArgs {
+  const int32_t *lo_in, *hi_in;   // [Lb] caller's ranges of the block's queries
+  int *lo, *hi;                   // [Lb] clamped (an invalid or empty range becomes lo = hi)
+  int *grp_tile0, *grp_start;     // as IndexerArgs
+  unsigned *status;
+  int Lb, QG, N;
+};
+cudaError_t launch_range_plan(const RangePlanArgs &a, cudaStream_t stream);
 
 cudaError_t launch_indexer(const CUtensorMap &tq, const CUtensorMap &tk, const IndexerArgs &a, int D_I, int H_I,
                            bool fp8, bool pilot, int grid, cudaStream_t stream);
@@ -47,6 +66,8 @@ struct SelectArgs {
   int32_t *topk_idx;              // [L, topk] whole chunk
   float *topk_score;              // [L, topk] or nullptr
   int dense_ld, n_samples, cap, fb_slots;
+  const int *key_lo, *key_hi;     // [Lb] clamped per-query ranges, or nullptr (causal)
+  int sample_stride;              // with ranges: pilot sample i is key i * sample_stride
   int t0, Lb, q_pos0;             // block: first query (chunk row), size, position of first query
   int N, H_I, D_I, topk, fp8;
 };

@@ -93,6 +93,7 @@ __device__ __forceinline__ float threshold_float(unsigned key) {
 
 // Per-group number of 128-key tiles.
 __device__ __forceinline__ int idx_group_tiles(const IndexerArgs &a, int g, int QG) {
+  if (!a.pilot && a.grp_start != nullptr) return a.grp_start[g + 1] - a.grp_start[g];
   int keys;
   if (a.pilot) {
     keys = a.n_keys;
@@ -103,17 +104,34 @@ __device__ __forceinline__ int idx_group_tiles(const IndexerArgs &a, int g, int 
   return (keys + 127) / 128;
 }
 
-// Tile range of this CTA in the linearised (group, key tile) space.
+// First 128-key tile of group g (per-query ranges only; 0 otherwise).
+__device__ __forceinline__ int idx_group_tile0(const IndexerArgs &a, int g) {
+  return (!a.pilot && a.grp_start != nullptr) ? a.grp_tile0[g] : 0;
+}
+
+// Tile range of this CTA in the linearised (group, key tile) space.  `key0`
+// is the first key of the current tile.
 struct TileCursor {
-  int g, tile, ntiles_g, left;
+  int g, tile, ntiles_g, left, tile0;
+  __device__ __forceinline__ int key0() const { return (tile0 + tile) * 128; }
 };
 
 __device__ __forceinline__ TileCursor idx_cursor_begin(const IndexerArgs &a, int QG) {
-  const long long T = a.total_tiles;
+  const int G = (a.Lb + QG - 1) / QG;
+  const long long T = (!a.pilot && a.grp_start != nullptr) ? a.grp_start[G] : a.total_tiles;
   const long long u0 = T * blockIdx.x / gridDim.x;
   const long long u1 = T * (blockIdx.x + 1) / gridDim.x;
   TileCursor c;
   c.left = static_cast<int>(u1 - u0);
+  c.g = 0;
+  c.tile = 0;
+  c.ntiles_g = 0;
+  c.tile0 = 0;
+  if (c.left <= 0) {
+    c.left = 0;
+    return c;
+  }
+  // u0 < T, so the walk stops at a group that has tiles (empty groups are passed over).
   long long acc = 0;
   int g = 0;
   int nt = idx_group_tiles(a, 0, QG);
@@ -125,6 +143,7 @@ __device__ __forceinline__ TileCursor idx_cursor_begin(const IndexerArgs &a, int
   c.g = g;
   c.tile = static_cast<int>(u0 - acc);
   c.ntiles_g = nt;
+  c.tile0 = idx_group_tile0(a, g);
   return c;
 }
 
@@ -132,8 +151,13 @@ __device__ __forceinline__ void idx_cursor_next(TileCursor &c, const IndexerArgs
   --c.left;
   if (++c.tile == c.ntiles_g) {
     c.tile = 0;
-    ++c.g;
-    c.ntiles_g = idx_group_tiles(a, c.g, QG);
+    if (c.left <= 0) return;  // nothing follows; do not look past the last group
+    // tiles remain, so a later group has some
+    do {
+      ++c.g;
+      c.ntiles_g = idx_group_tiles(a, c.g, QG);
+    } while (c.ntiles_g == 0);
+    c.tile0 = idx_group_tile0(a, c.g);
   }
 }
 
@@ -214,7 +238,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
         mbar_arrive_expect_tx(&full[stage], C::K_TILE);
         for (int at = 0; at < C::ATOMS; ++at)
           tma_load_2d(k_s + stage * C::K_TILE + at * C::BM * 128, &tmap_k, &full[stage], at * C::ATOM_ELEMS,
-                      c.tile * C::BM);
+                      c.key0());
         ++issued;
         if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         idx_cursor_next(c, a, C::QG);
@@ -304,6 +328,9 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     const unsigned lane_mask_lt = (1u << lane) - 1u;
     float *w_w = w_s + ew * C::COLS;   // this warp's head weights: [QH queries][HI]
     float *tau_w = tau_s + ew * C::COLS;
+    int *lo_w = reinterpret_cast<int *>(tau_w + QH);      // per-query key ranges (ranges mode)
+    int *hi_w = reinterpret_cast<int *>(tau_w + 2 * QH);
+    static_assert(3 * C::QH <= C::COLS, "thresholds and ranges share the per-warp slot");
     unsigned long long *stg = reinterpret_cast<unsigned long long *>(smem + C::OFF_STG) + ew * QH * SB;
     int cnt[QH];                   // staged candidates per query (warp-uniform)
 #pragma unroll
@@ -344,6 +371,10 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
           for (int j = lane; j < QH; j += 32) {
             const int tl = g * C::QG + slot * QH + j;
             tau_w[j] = (tl < a.Lb) ? threshold_float(a.tau[tl]) : INFINITY;
+            if (a.key_lo != nullptr) {
+              lo_w[j] = (tl < a.Lb) ? a.key_lo[tl] : 0;
+              hi_w[j] = (tl < a.Lb) ? a.key_hi[tl] : 0;
+            }
           }
         }
         __syncwarp();
@@ -353,7 +384,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
       tc_fence_after();
       const unsigned taddr =
           tmem_base + (static_cast<unsigned>(quarter * 32) << 16) + acc * 256 + slot * C::COLS;
-      const int key = c.tile * C::BM + quarter * 32 + lane;
+      const int key = c.key0() + quarter * 32 + lane;
       // One 32-column chunk of the accumulator at a time (keeps the live
       // register set small); the buffer goes back to the MMA warp after the
       // last chunk has been read.
@@ -387,7 +418,8 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
         if (PILOT) {
           if (tl < a.Lb && key < a.n_keys) a.dense[static_cast<long long>(tl) * a.dense_ld + key] = score;
         } else {
-          const bool pass = (tl < a.Lb) && (key <= a.q_pos0 + tl) && (score >= tau_w[qq]);
+          const bool vis = a.key_lo != nullptr ? (key >= lo_w[qq] && key < hi_w[qq]) : (key <= a.q_pos0 + tl);
+          const bool pass = (tl < a.Lb) && vis && (score >= tau_w[qq]);
           const unsigned m = __ballot_sync(0xffffffffu, pass);
           if (m) {
             const int n = __popc(m);

@@ -102,21 +102,29 @@ __global__ void __launch_bounds__(256) threshold_kernel(SelectArgs a) {
       a.fb_counters[1] = 0;
     }
   }
-  const int nvis = a.q_pos0 + tl + 1;
+  // Visible keys [lo, lo + nvis) and the pilot samples [i0, i0 + ns) among them.
+  int lo = 0, nvis = a.q_pos0 + tl + 1, i0 = 0, ns = a.n_samples;
+  if (a.key_lo != nullptr) {
+    lo = a.key_lo[tl];
+    nvis = a.key_hi[tl] - lo;
+    const int st = max(1, a.sample_stride);
+    i0 = min(a.n_samples, (lo + st - 1) / st);
+    ns = min(a.n_samples, (a.key_hi[tl] + st - 1) / st) - i0;
+  }
   const int need = min(a.topk, nvis);
   unsigned tau = 0u;  // key 0: every score passes
-  if (a.dense != nullptr && nvis > a.cap && a.n_samples > 0) {
+  if (a.dense != nullptr && nvis > a.cap && ns > 0) {
     const double z = 5.0;
-    const double x = static_cast<double>(need) * a.n_samples / nvis;
+    const double x = static_cast<double>(need) * ns / nvis;
     const double rt = z / 2.0 + sqrt(z * z / 4.0 + x);
     const double rd = ceil(rt * rt);
-    if (rd < a.n_samples) {
+    if (rd < ns) {
       const int r = static_cast<int>(rd);
-      const float *row = a.dense + static_cast<long long>(tl) * a.dense_ld;
-      for (int i = threadIdx.x; i < a.n_samples; i += blockDim.x) keys[i] = float_order_key(row[i]);
+      const float *row = a.dense + static_cast<long long>(tl) * a.dense_ld + i0;
+      for (int i = threadIdx.x; i < ns; i += blockDim.x) keys[i] = float_order_key(row[i]);
       __syncthreads();
       unsigned prefix, mask;
-      block_radix_select<unsigned>([&](int i) { return keys[i]; }, a.n_samples, r, prefix, mask, hist, misc);
+      block_radix_select<unsigned>([&](int i) { return keys[i]; }, ns, r, prefix, mask, hist, misc);
       tau = prefix;
     }
   }
@@ -183,7 +191,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   __shared__ int total, nsel;
   const int tl = blockIdx.x;
   const int t = a.t0 + tl;
-  const int nvis = a.q_pos0 + tl + 1;
+  const int lo = a.key_lo != nullptr ? a.key_lo[tl] : 0;  // visible keys [lo, lo + nvis)
+  const int nvis = a.key_lo != nullptr ? a.key_hi[tl] - lo : a.q_pos0 + tl + 1;
   const int need = min(a.topk, nvis);
   const int count = a.cand_count[tl];
   if (count > a.cap || count < need) {
@@ -214,7 +223,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     for (int i = threadIdx.x; i < count; i += blockDim.x) {
       const unsigned long long k = fetch(i);
       if (k >= prefix) {
-        const unsigned idx = ~static_cast<unsigned>(k & 0xFFFFFFFFull);
+        const unsigned idx = ~static_cast<unsigned>(k & 0xFFFFFFFFull) - static_cast<unsigned>(lo);
         atomicOr(&bitmap[idx >> 5], 1u << (idx & 31));
       }
     }
@@ -229,7 +238,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
       while (bits) {
         const int b = __ffs(bits) - 1;
         bits &= bits - 1;
-        if (pos < need) out[pos] = wd * 32 + b;
+        if (pos < need) out[pos] = lo + wd * 32 + b;
         ++pos;
       }
     }
@@ -299,13 +308,15 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(SelectArgs a) {
     if (job >= *reinterpret_cast<volatile int *>(&a.fb_counters[0])) break;
     const int tl = a.fb_list[job];
     const int t = a.t0 + tl;
-    const int nvis = a.q_pos0 + tl + 1;
+    const int lo = a.key_lo != nullptr ? a.key_lo[tl] : 0;  // visible keys [lo, lo + nvis)
+    const int nvis = a.key_lo != nullptr ? a.key_hi[tl] - lo : a.q_pos0 + tl + 1;
     const int need = min(a.topk, nvis);
     for (int i = threadIdx.x; i < a.H_I * a.D_I; i += blockDim.x)
       q_s[i] = idx_elem(a.q_idx, static_cast<long long>(t) * a.H_I * a.D_I + i, a.fp8);
     for (int i = threadIdx.x; i < a.H_I; i += blockDim.x) w_s[i] = a.w[static_cast<long long>(t) * a.H_I + i];
     __syncthreads();
-    for (int s = threadIdx.x; s < nvis; s += blockDim.x) {
+    for (int j = threadIdx.x; j < nvis; j += blockDim.x) {
+      const int s = lo + j;
       float kr[128];
       for (int d = 0; d < a.D_I; ++d) kr[d] = idx_elem(a.k_idx, static_cast<long long>(s) * a.D_I + d, a.fp8);
       float score = 0.0f;
@@ -314,12 +325,13 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(SelectArgs a) {
         for (int d = 0; d < a.D_I; ++d) dot = fmaf(q_s[h * a.D_I + d], kr[d], dot);
         score = fmaf(w_s[h], fmaxf(dot, 0.0f), score);
       }
-      scores[s] = score;
+      scores[j] = score;
     }
     __syncthreads();
-    auto key_of = [&](int s) {
-      return (static_cast<unsigned long long>(float_order_key(scores[s])) << 32) |
-             static_cast<unsigned>(~static_cast<unsigned>(s));
+    // j indexes the visible keys; key lo + j breaks ties
+    auto key_of = [&](int j) {
+      return (static_cast<unsigned long long>(float_order_key(scores[j])) << 32) |
+             static_cast<unsigned>(~static_cast<unsigned>(lo + j));
     };
     unsigned long long prefix = 0, mask = 0;
     if (nvis > need) block_radix_select<unsigned long long>(key_of, nvis, need, prefix, mask, hist, misc);
@@ -345,7 +357,7 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(SelectArgs a) {
       if (sel) {
         const int pos = base_s + warp_off[warp] + __popc(bal & ((1u << lane) - 1u));
         if (pos < need) {
-          out[pos] = s;
+          out[pos] = lo + s;
           if (osc) osc[pos] = scores[s];
         }
       }
@@ -359,6 +371,58 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(SelectArgs a) {
       if (osc) osc[j] = -INFINITY;
     }
   }
+}
+
+// ------------------------------------------------------------------ range plan
+// Per-query key ranges: clamp each into [0, N] (a range with lo < 0, hi > N
+// or lo > hi is flagged and made empty), then give every query group the
+// window of 128-key tiles that covers its queries' non-empty ranges, and the
+// exclusive prefix of the windows' sizes for the indexer's work split.
+__global__ void __launch_bounds__(128) range_plan_kernel(RangePlanArgs a) {
+  __shared__ int cnt_s[128];
+  const int G = (a.Lb + a.QG - 1) / a.QG;
+  for (int t = threadIdx.x; t < a.Lb; t += blockDim.x) {
+    int lo = a.lo_in[t], hi = a.hi_in[t];
+    if (lo < 0 || hi > a.N || lo > hi) {
+      atomicOr(a.status, DEV_BAD_INDEX);
+      lo = hi = 0;
+    }
+    a.lo[t] = lo;
+    a.hi[t] = hi;
+  }
+  __syncthreads();
+  const int g = threadIdx.x;
+  int n = 0, t0 = 0;
+  if (g < G) {
+    int mn = a.N, mx = 0;
+    for (int t = g * a.QG; t < min(a.Lb, (g + 1) * a.QG); ++t) {
+      if (a.lo[t] < a.hi[t]) {
+        mn = min(mn, a.lo[t]);
+        mx = max(mx, a.hi[t]);
+      }
+    }
+    if (mx > mn) {
+      t0 = mn / 128;
+      n = (mx + 127) / 128 - t0;
+    }
+    a.grp_tile0[g] = t0;
+  }
+  cnt_s[threadIdx.x] = n;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int i = 0; i < G; ++i) {
+      a.grp_start[i] = acc;
+      acc += cnt_s[i];
+    }
+    a.grp_start[G] = acc;
+  }
+}
+
+cudaError_t launch_range_plan(const RangePlanArgs &a, cudaStream_t stream) {
+  if ((a.Lb + a.QG - 1) / a.QG > 128) return cudaErrorInvalidValue;
+  range_plan_kernel<<<1, 128, 0, stream>>>(a);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ pack plan

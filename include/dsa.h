@@ -122,6 +122,29 @@ dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float 
  *     overlap on the GPU (two streams, two host threads) race on the array
  *     and must be serialised by the caller.
  */
+/*
+ * dsa_indexer_topk with general visibility carried by an index mask instead of
+ * the causal triangle (llama.cpp PR #25917, discussion: causality applied to
+ * the indices, so that a unified cache holding several sequences, or a
+ * non-triangular mask, can be expressed per query).  Query t sees exactly the
+ * keys s with key_lo[t] <= s < key_hi[t]; its top-k is taken among them, with
+ * -1 padding when the range holds fewer than topk keys (an empty range
+ * selects nothing).  Everything else as dsa_indexer_topk.
+ *
+ *   key_lo, key_hi [L] int32, device, 4-byte aligned; 0 <= key_lo[t] <=
+ *                  key_hi[t] <= N.  A range that breaks this is treated as
+ *                  empty and flags the device status word (bit 1, see
+ *                  dsa_workspace_status).
+ *
+ * Packed sequences (batched prefill): with several sequences stored one after
+ * another in the cache, query t of the sequence starting at key b sees
+ * [b, its own position + 1).  Workspace: dsa_indexer_topk_workspace.
+ */
+dsa_status_t dsa_indexer_topk_ranges(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
+                                     int L, int N, int H_I, int D_I, const int32_t *key_lo,
+                                     const int32_t *key_hi, int topk, int32_t *topk_idx, float *topk_score,
+                                     void *workspace, size_t workspace_bytes, dsa_stream_t stream);
+
 dsa_status_t dsa_indexer_topk_noalloc(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
                                       int L, int N, int H_I, int D_I, int q_pos0, int topk, int32_t *topk_idx,
                                       float *topk_score, dsa_stream_t stream);
@@ -184,6 +207,17 @@ dsa_status_t dsa_prefill_chunk(const void *q_idx, const void *k_idx, const float
                                const void *q, const void *kv, int L, int N, int H_I, int D_I, int H, int q_pos0,
                                int topk, float scale, int query_block, int32_t *topk_idx_out, void *out, float *lse,
                                void *workspace, size_t workspace_bytes, dsa_stream_t stream);
+
+/*
+ * dsa_prefill_chunk with general visibility: query t sees keys key_lo[t] <=
+ * s < key_hi[t] (as dsa_indexer_topk_ranges) instead of the causal prefix
+ * from q_pos0.  Workspace: dsa_prefill_chunk_workspace.
+ */
+dsa_status_t dsa_prefill_chunk_ranges(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
+                                      const void *q, const void *kv, int L, int N, int H_I, int D_I, int H,
+                                      const int32_t *key_lo, const int32_t *key_hi, int topk, float scale,
+                                      int query_block, int32_t *topk_idx_out, void *out, float *lse,
+                                      void *workspace, size_t workspace_bytes, dsa_stream_t stream);
 
 /*
  * dsa_prefill_chunk, additionally recording CUDA events on `stream` between
