@@ -91,9 +91,11 @@ __device__ __forceinline__ float threshold_float(unsigned key) {
   return key < 0x00800000u ? -INFINITY : order_key_float(key);
 }
 
-// Per-group number of 128-key tiles.
+// Per-group number of 128-key tiles.  RANGES: per-query key ranges (the
+// planned windows); otherwise the causal prefix (or, in PILOT mode, all samples).
+template <bool RANGES>
 __device__ __forceinline__ int idx_group_tiles(const IndexerArgs &a, int g, int QG) {
-  if (!a.pilot && a.grp_start != nullptr) return a.grp_start[g + 1] - a.grp_start[g];
+  if (RANGES) return a.grp_start[g + 1] - a.grp_start[g];
   int keys;
   if (a.pilot) {
     keys = a.n_keys;
@@ -105,8 +107,9 @@ __device__ __forceinline__ int idx_group_tiles(const IndexerArgs &a, int g, int 
 }
 
 // First 128-key tile of group g (per-query ranges only; 0 otherwise).
+template <bool RANGES>
 __device__ __forceinline__ int idx_group_tile0(const IndexerArgs &a, int g) {
-  return (!a.pilot && a.grp_start != nullptr) ? a.grp_tile0[g] : 0;
+  return RANGES ? a.grp_tile0[g] : 0;
 }
 
 // Tile range of this CTA in the linearised (group, key tile) space.  `key0`
@@ -116,9 +119,10 @@ struct TileCursor {
   __device__ __forceinline__ int key0() const { return (tile0 + tile) * 128; }
 };
 
+template <bool RANGES>
 __device__ __forceinline__ TileCursor idx_cursor_begin(const IndexerArgs &a, int QG) {
   const int G = (a.Lb + QG - 1) / QG;
-  const long long T = (!a.pilot && a.grp_start != nullptr) ? a.grp_start[G] : a.total_tiles;
+  const long long T = RANGES ? a.grp_start[G] : a.total_tiles;
   const long long u0 = T * blockIdx.x / gridDim.x;
   const long long u1 = T * (blockIdx.x + 1) / gridDim.x;
   TileCursor c;
@@ -134,19 +138,20 @@ __device__ __forceinline__ TileCursor idx_cursor_begin(const IndexerArgs &a, int
   // u0 < T, so the walk stops at a group that has tiles (empty groups are passed over).
   long long acc = 0;
   int g = 0;
-  int nt = idx_group_tiles(a, 0, QG);
+  int nt = idx_group_tiles<RANGES>(a, 0, QG);
   while (acc + nt <= u0) {
     acc += nt;
     ++g;
-    nt = idx_group_tiles(a, g, QG);
+    nt = idx_group_tiles<RANGES>(a, g, QG);
   }
   c.g = g;
   c.tile = static_cast<int>(u0 - acc);
   c.ntiles_g = nt;
-  c.tile0 = idx_group_tile0(a, g);
+  c.tile0 = idx_group_tile0<RANGES>(a, g);
   return c;
 }
 
+template <bool RANGES>
 __device__ __forceinline__ void idx_cursor_next(TileCursor &c, const IndexerArgs &a, int QG) {
   --c.left;
   if (++c.tile == c.ntiles_g) {
@@ -155,13 +160,13 @@ __device__ __forceinline__ void idx_cursor_next(TileCursor &c, const IndexerArgs
     // tiles remain, so a later group has some
     do {
       ++c.g;
-      c.ntiles_g = idx_group_tiles(a, c.g, QG);
+      c.ntiles_g = idx_group_tiles<RANGES>(a, c.g, QG);
     } while (c.ntiles_g == 0);
-    c.tile0 = idx_group_tile0(a, c.g);
+    c.tile0 = idx_group_tile0<RANGES>(a, c.g);
   }
 }
 
-template <int DI, int HI, bool FP8, bool PILOT>
+template <int DI, int HI, bool FP8, bool PILOT, bool RANGES>
 __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    IndexerArgs a) {
@@ -217,7 +222,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      TileCursor c = idx_cursor_begin(a, C::QG);
+      TileCursor c = idx_cursor_begin<RANGES>(a, C::QG);
       int stage = 0;
       unsigned phase = 0, qphase = 0;
       int prev_g = -1, issued = 0, q_issued = 0;
@@ -241,7 +246,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
                       c.key0());
         ++issued;
         if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
-        idx_cursor_next(c, a, C::QG);
+        idx_cursor_next<RANGES>(c, a, C::QG);
       }
       if (!ok) {
         atomicOr(a.status, DEV_TIMEOUT);
@@ -259,7 +264,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    TileCursor c = idx_cursor_begin(a, C::QG);
+    TileCursor c = idx_cursor_begin<RANGES>(a, C::QG);
     constexpr unsigned idesc = make_idesc(C::BM, C::BN, FP8 ? 0u : 1u, 0u, 0u);
     int stage = 0, acc = 0, prev_g = -1;
     unsigned phase = 0, acc_phase = 0, qphase = 0;
@@ -275,7 +280,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
       if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
       tc_fence_after();
       TileCursor nx = c;
-      idx_cursor_next(nx, a, C::QG);
+      idx_cursor_next<RANGES>(nx, a, C::QG);
       const bool last_of_group = (nx.left == 0) || (nx.g != g);
       if (lane == 0) {
         const unsigned d_tmem = tmem_base + acc * 256;
@@ -321,7 +326,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     const int slot = ew >> 2;         // which 64 accumulator columns
     constexpr int QH = C::QH;         // queries per warp
     constexpr int SB = C::SB;
-    TileCursor c = idx_cursor_begin(a, C::QG);
+    TileCursor c = idx_cursor_begin<RANGES>(a, C::QG);
     int acc = 0, prev_g = -1;
     unsigned acc_phase = 0;
     bool ok = true;
@@ -371,7 +376,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
           for (int j = lane; j < QH; j += 32) {
             const int tl = g * C::QG + slot * QH + j;
             tau_w[j] = (tl < a.Lb) ? threshold_float(a.tau[tl]) : INFINITY;
-            if (a.key_lo != nullptr) {
+            if (RANGES) {
               lo_w[j] = (tl < a.Lb) ? a.key_lo[tl] : 0;
               hi_w[j] = (tl < a.Lb) ? a.key_hi[tl] : 0;
             }
@@ -418,7 +423,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
         if (PILOT) {
           if (tl < a.Lb && key < a.n_keys) a.dense[static_cast<long long>(tl) * a.dense_ld + key] = score;
         } else {
-          const bool vis = a.key_lo != nullptr ? (key >= lo_w[qq] && key < hi_w[qq]) : (key <= a.q_pos0 + tl);
+          const bool vis = RANGES ? (key >= lo_w[qq] && key < hi_w[qq]) : (key <= a.q_pos0 + tl);
           const bool pass = (tl < a.Lb) && vis && (score >= tau_w[qq]);
           const unsigned m = __ballot_sync(0xffffffffu, pass);
           if (m) {
@@ -435,7 +440,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
       }
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-      idx_cursor_next(c, a, C::QG);
+      idx_cursor_next<RANGES>(c, a, C::QG);
     }
     if (ok && !PILOT && prev_g >= 0) {
 #pragma unroll
@@ -455,11 +460,11 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
   }
 }
 
-template <int DI, int HI, bool FP8, bool PILOT>
+template <int DI, int HI, bool FP8, bool PILOT, bool RANGES>
 static cudaError_t launch_indexer_t(const CUtensorMap &tq, const CUtensorMap &tk, const IndexerArgs &a, int grid,
                                     cudaStream_t stream) {
   using C = IdxCfg<DI, HI, FP8>;
-  auto kern = indexer_kernel<DI, HI, FP8, PILOT>;
+  auto kern = indexer_kernel<DI, HI, FP8, PILOT, RANGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, a);
@@ -472,8 +477,9 @@ cudaError_t launch_indexer(const CUtensorMap &tq, const CUtensorMap &tk, const I
                            bool fp8, bool pilot, int grid, cudaStream_t stream) {
 #define DSA_IDX_CASE(DI_, HI_, FP8_)                                                            \
   if (D_I == DI_ && H_I == HI_ && fp8 == FP8_)                                                  \
-    return pilot ? launch_indexer_t<DI_, HI_, FP8_, true>(tq, tk, a, grid, stream)              \
-                 : launch_indexer_t<DI_, HI_, FP8_, false>(tq, tk, a, grid, stream);
+    return pilot            ? launch_indexer_t<DI_, HI_, FP8_, true, false>(tq, tk, a, grid, stream)  \
+           : a.key_lo != nullptr ? launch_indexer_t<DI_, HI_, FP8_, false, true>(tq, tk, a, grid, stream) \
+                             : launch_indexer_t<DI_, HI_, FP8_, false, false>(tq, tk, a, grid, stream);
   DSA_IDX_CASE(128, 32, false)
   DSA_IDX_CASE(128, 32, true)
   DSA_IDX_CASE(64, 4, false)
