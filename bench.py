@@ -375,6 +375,57 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         torch.distributed.destroy_process_group()
 
 
+def run_crossover(args) -> None:
+    """Dense-vs-sparse crossover (measurement only, one JSON line per context length).
+
+    For a 1,024-query chunk at the end of an N-key cache (the 128K workload's
+    distributions, k = 2,048, 64 heads): the whole sparse path
+    (dsa_prefill_chunk) against dense causal attention over every visible key,
+    run through the same tcgen05 attention kernel with all visible keys
+    selected.  CUDA events, L2 flushed before every timed call.
+    """
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    import deepseek_sparse_attention_relu_b200 as dsa
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps=5, warm=3):
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    for N in (2048, 4096, 8192, 16384, 32768, 65536, 131072):
+        L = 1024
+        cfg = dsa_inputs.small_variant(dsa_inputs.CTX128K, N=N, L=L, topk=2048, H=64)
+        g = {k: v.to(dev) for k, v in dsa_inputs.generate(cfg).items()}
+        out = torch.empty(L, cfg.H, 512, dtype=torch.bfloat16, device=dev)
+        ws = dsa.alloc_workspace(dsa.dsa_prefill_chunk_workspace(L, N, cfg.H_I, cfg.D_I, cfg.H, cfg.topk, 0,
+                                                                 dsa.DSA_BF16, False), dev)
+        sparse_ms = timed(lambda: dsa.dsa_prefill_chunk(g["q_idx"], g["k_idx"], g["w"], g["q"], g["kv"],
+                                                        cfg.q_pos0, cfg.topk, cfg.scale, out, workspace=ws))
+        # every visible key of query t: 0 .. q_pos0 + t, then -1
+        ar = torch.arange(N, dtype=torch.int32, device=dev)
+        vis = (cfg.q_pos0 + torch.arange(L, device=dev)).unsqueeze(1)
+        dense_idx = torch.where(ar.unsqueeze(0) <= vis, ar.unsqueeze(0), torch.full_like(ar.unsqueeze(0), -1))
+        dense_idx = dense_idx.to(torch.int32).contiguous()
+        wsd = dsa.alloc_workspace(dsa.dsa_sparse_mla_workspace(L, cfg.H, N), dev)
+        dense_ms = timed(lambda: dsa.dsa_sparse_mla_prefill(g["q"], g["kv"], dense_idx, cfg.scale, out,
+                                                            workspace=wsd))
+        print(json.dumps({"crossover": True, "N": N, "L": L, "topk": cfg.topk, "H": cfg.H,
+                          "sparse_path_ms": round(sparse_ms, 4), "dense_attention_ms": round(dense_ms, 4),
+                          "dense_over_sparse": round(dense_ms / sparse_ms, 3)}), flush=True)
+        del g, out, ws, wsd, dense_idx
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -383,6 +434,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=dsa_inputs.CTX128K.name, choices=sorted(dsa_inputs.BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--crossover", action="store_true",
+                    help="measure the dense-vs-sparse crossover instead (JSON line per context length)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -391,7 +444,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         log(f"[bench] note: WORLD_SIZE={world} but --gpus={args.gpus}; using WORLD_SIZE")
-    if args.impl == "reference":
+    if args.crossover:
+        if rank == 0:
+            run_crossover(args)
+    elif args.impl == "reference":
         run_reference(args, rank, world)
     else:
         run_ours(args, rank, world, local_rank)
