@@ -107,3 +107,21 @@ def test_topk_one_and_topk_equals_visible():
         inp = dsa_inputs.generate(cfg, with_mla=False)
         idx, _ = run_indexer(cfg, inp)
         check_rows(cfg, inp, idx, range(cfg.L))
+
+
+# Every indexer shape the header declares supported, on the pilot path with a ragged query count:
+# (D_I, H_I, fp8).  The five workloads only reach (128, 32, *) and (64, 4, bf16).
+OTHER_SHAPES = [(128, 16, False), (128, 16, True), (128, 8, False), (128, 8, True), (64, 32, False)]
+
+
+@pytest.mark.parametrize("D_I,H_I,fp8", OTHER_SHAPES, ids=[f"D{d}-H{h}-{'fp8' if f else 'bf16'}"
+                                                          for d, h, f in OTHER_SHAPES])
+def test_supported_indexer_shapes(D_I, H_I, fp8):
+    from dataclasses import replace
+    base = dsa_inputs.CTX64K if fp8 else dsa_inputs.CTX128K
+    cfg = replace(dsa_inputs.small_variant(base, N=20000, L=141, topk=512), H_I=H_I, D_I=D_I,
+                  name=f"shape-D{D_I}-H{H_I}-{'fp8' if fp8 else 'bf16'}")
+    inp = dsa_inputs.generate(cfg, with_mla=False)
+    assert tuple(inp["q_idx"].shape) == (cfg.L, H_I, D_I)
+    idx, sc = run_indexer(cfg, inp, with_scores=True)
+    check_rows(cfg, inp, idx, list(range(0, cfg.L, 7)) + [cfg.L - 1], gpu_scores=sc)
