@@ -23,6 +23,12 @@
 //     double-buffered with the stages at no extra shared memory;
 //   * O += P V on tcgen05 (M = 64, N = 2 x 256 latent columns, K = 64 keys),
 //     V read in place from the gathered tile as an MN-major operand.
+// The producers also pull the next tile's rows from HBM into L2
+// (prefetch.global.L2) while the current tile's copies land, and the MMA warp
+// polls its barriers with the non-suspending mbarrier.test_wait.  Split-key
+// mode (chunks with few queries, e.g. decode): CTA z of a query attends its
+// z-th share of the selection and writes a normalised fp32 partial and its
+// log-sum-exp; mla_combine_kernel merges the shares.
 // TMEM: the two 64 x 256 fp32 halves of O sit in the two half-subpartitions
 // (lanes 0-15 and 16-31 of each 32-lane quarter) of columns 0-255, the two S
 // buffers in columns 256-383.  Warp roles: warp 0 MMA issuer / TMEM owner,
