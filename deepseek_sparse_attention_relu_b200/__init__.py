@@ -27,7 +27,8 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 EXPORTED = ("dsa_version", "dsa_status_string", "dsa_last_error_string", "dsa_indexer_topk_workspace", "dsa_indexer_topk",
             "dsa_sparse_mla_workspace", "dsa_sparse_mla_prefill", "dsa_prefill_chunk_workspace",
             "dsa_prefill_chunk", "dsa_prefill_chunk_profiled", "dsa_workspace_status",
-            "dsa_indexer_topk_noalloc", "dsa_indexer_topk_ranges", "dsa_prefill_chunk_ranges")
+            "dsa_indexer_topk_noalloc", "dsa_indexer_topk_ranges", "dsa_prefill_chunk_ranges",
+            "dsa_selftest_wait_timeout")
 
 _lib = None
 
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_indexer_topk_ranges.argtypes = [P, P, P, I, I, I, I, I, P, P, I, P, P, P, Z, P]
         L.dsa_prefill_chunk_ranges.restype = I
         L.dsa_prefill_chunk_ranges.argtypes = [P, P, P, I, P, P, I, I, I, I, I, P, P, I, F, I, P, P, P, P, Z, P]
+        L.dsa_selftest_wait_timeout.restype = I
+        L.dsa_selftest_wait_timeout.argtypes = [P, Z, ctypes.c_uint, P]
         L.dsa_workspace_status.restype = I
         L.dsa_workspace_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint)]
         _lib = L
@@ -283,6 +286,12 @@ def dsa_prefill_chunk_profiled(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torc
         _dev(lse, "lse", (torch.float32,)), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream), handles, len(events)),
         "dsa_prefill_chunk_profiled")
+
+
+def dsa_selftest_wait_timeout(workspace: torch.Tensor, limit_ms: int = 50, stream=None) -> None:
+    """Run the bounded-wait self-test into `workspace` (see include/dsa.h); read it with dsa_workspace_status."""
+    _check(lib().dsa_selftest_wait_timeout(_dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                                           int(limit_ms), _stream(stream)), "dsa_selftest_wait_timeout")
 
 
 def dsa_workspace_status(workspace: torch.Tensor, stream=None) -> int:

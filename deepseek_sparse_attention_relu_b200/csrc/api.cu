@@ -665,6 +665,18 @@ dsa_status_t dsa_prefill_chunk_profiled(const void *q_idx, const void *k_idx, co
                             reinterpret_cast<cudaEvent_t *>(const_cast<void **>(events)), n_events);
 }
 
+dsa_status_t dsa_selftest_wait_timeout(void *workspace, size_t workspace_bytes, unsigned limit_ms,
+                                       dsa_stream_t stream_) {
+  if (workspace == nullptr || workspace_bytes < kHeaderBytes) return DSA_ERR_WORKSPACE;
+  if (limit_ms == 0 || limit_ms > 2000) return DSA_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  unsigned *status = static_cast<unsigned *>(workspace);
+  if (!cuda_ok(cudaMemsetAsync(status, 0, kHeaderBytes, stream))) return DSA_ERR_CUDA;
+  return cuda_ok(launch_wait_timeout_probe(status, static_cast<unsigned long long>(limit_ms) * 1000000ull, stream))
+             ? DSA_OK
+             : DSA_ERR_CUDA;
+}
+
 dsa_status_t dsa_workspace_status(const void *workspace, dsa_stream_t stream_, unsigned *flags) {
   if (workspace == nullptr || flags == nullptr) return DSA_ERR_INVALID_ARG;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);

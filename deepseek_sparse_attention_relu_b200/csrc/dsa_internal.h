@@ -44,6 +44,7 @@ struct RangePlanArgs {
   int Lb, QG, N;
 };
 cudaError_t launch_range_plan(const RangePlanArgs &a, cudaStream_t stream);
+cudaError_t launch_wait_timeout_probe(unsigned *status, unsigned long long limit_ns, cudaStream_t stream);
 
 cudaError_t launch_indexer(const CUtensorMap &tq, const CUtensorMap &tk, const IndexerArgs &a, int D_I, int H_I,
                            bool fp8, bool pilot, int grid, cudaStream_t stream);

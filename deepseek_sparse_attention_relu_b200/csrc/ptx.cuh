@@ -86,7 +86,8 @@ __device__ __forceinline__ void prefetch_l2_line(const void *p) {
 // Wait for the phase with the given parity to complete.  Returns false after
 // the wall-clock limit, or as soon as *abort becomes non-zero (another role of
 // the CTA gave up; pass nullptr to ignore it); the caller then unwinds.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity, volatile int *abort) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, unsigned parity, volatile int *abort,
+                                                unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = globaltimer();
   unsigned spins = 0;
@@ -94,9 +95,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     if (((++spins) & 63u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) return false;
+      if (globaltimer() - t0 > limit_ns) return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity, volatile int *abort) {
+  return mbar_wait_limit(bar, parity, abort, kWaitLimitNs);
 }
 
 // mbar_wait for a whole warp: lane 0 polls, the others wait at the warp

@@ -373,6 +373,23 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(SelectArgs a) {
   }
 }
 
+// ------------------------------------------------------------------ wait self-test
+// The bounded-wait path of every kernel, exercised on purpose: one thread
+// waits on an mbarrier that nothing arrives on, gives up after limit_ns and
+// records DEV_TIMEOUT, exactly as a kernel whose producer stalled would.
+__global__ void wait_timeout_probe_kernel(unsigned *status, unsigned long long limit_ns) {
+  __shared__ uint64_t never;
+  if (threadIdx.x != 0) return;
+  mbar_init(&never, 1);
+  fence_mbar_init();
+  if (!mbar_wait_limit(&never, 0u, nullptr, limit_ns)) atomicOr(status, DEV_TIMEOUT);
+}
+
+cudaError_t launch_wait_timeout_probe(unsigned *status, unsigned long long limit_ns, cudaStream_t stream) {
+  wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ range plan
 // Per-query key ranges: clamp each into [0, N] (a range with lo < 0, hi > N
 // or lo > hi is flagged and made empty), then give every query group the

@@ -234,6 +234,19 @@ dsa_status_t dsa_prefill_chunk_profiled(const void *q_idx, const void *k_idx, co
                                         dsa_stream_t stream, void *const *events, int n_events);
 
 /*
+ * Diagnostic with no counterpart in the method: exercises the bounded-wait
+ * error path that every kernel of this library takes when a wait on another
+ * role (or another block of the pipeline) never completes.  Clears the
+ * workspace's status word, then launches one thread that waits on an mbarrier
+ * nothing arrives on; after limit_ms (1..2000) it gives up and sets bit 0
+ * (timeout) of the status word, the context staying usable.  Read the result
+ * with dsa_workspace_status (expect DSA_ERR_INTERNAL with bit 0 set).
+ *   workspace: any workspace of this library (>= its 256-byte header).
+ */
+dsa_status_t dsa_selftest_wait_timeout(void *workspace, size_t workspace_bytes, unsigned limit_ms,
+                                       dsa_stream_t stream);
+
+/*
  * Synchronise `stream`, read the device status word at the start of a
  * workspace used by the calls above and store it in *flags (bit 0: a wait
  * timed out, bit 1: an index outside [0, N) reached the attention stage,
