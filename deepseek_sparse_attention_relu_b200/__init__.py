@@ -60,23 +60,26 @@ def lib() -> ctypes.CDLL:
         L.dsa_indexer_topk_workspace.restype = Z
         L.dsa_indexer_topk_workspace.argtypes = [I, I, I, I, I, I]
         L.dsa_indexer_topk.restype = I
-        L.dsa_indexer_topk.argtypes = [P, P, P, I, I, I, I, I, I, I, P, P, P, Z, P]
+        LL = ctypes.c_longlong
+        L.dsa_indexer_topk.argtypes = [P, P, LL, P, I, I, I, I, I, I, I, P, P, P, Z, P]
         L.dsa_sparse_mla_workspace.restype = Z
         L.dsa_sparse_mla_workspace.argtypes = [I, I, I]
         L.dsa_sparse_mla_prefill.restype = I
-        L.dsa_sparse_mla_prefill.argtypes = [P, P, P, I, I, I, I, F, P, P, P, Z, P]
+        L.dsa_sparse_mla_prefill.argtypes = [P, P, LL, P, I, I, I, I, F, P, P, P, Z, P]
         L.dsa_prefill_chunk_workspace.restype = Z
         L.dsa_prefill_chunk_workspace.argtypes = [I, I, I, I, I, I, I, I, I]
         L.dsa_prefill_chunk.restype = I
-        L.dsa_prefill_chunk.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, I, P, P, P, P, Z, P]
+        L.dsa_prefill_chunk.argtypes = [P, P, LL, P, I, P, P, LL, I, I, I, I, I, I, I, F, I, P, P, P, P, Z, P]
         L.dsa_prefill_chunk_profiled.restype = I
-        L.dsa_prefill_chunk_profiled.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, I, P, P, P, P, Z, P, P, I]
+        L.dsa_prefill_chunk_profiled.argtypes = [P, P, LL, P, I, P, P, LL, I, I, I, I, I, I, I, F, I, P, P, P, P, Z,
+                                                 P, P, I]
         L.dsa_indexer_topk_noalloc.restype = I
-        L.dsa_indexer_topk_noalloc.argtypes = [P, P, P, I, I, I, I, I, I, I, P, P, P]
+        L.dsa_indexer_topk_noalloc.argtypes = [P, P, LL, P, I, I, I, I, I, I, I, P, P, P]
         L.dsa_indexer_topk_ranges.restype = I
-        L.dsa_indexer_topk_ranges.argtypes = [P, P, P, I, I, I, I, I, P, P, I, P, P, P, Z, P]
+        L.dsa_indexer_topk_ranges.argtypes = [P, P, LL, P, I, I, I, I, I, P, P, I, P, P, P, Z, P]
         L.dsa_prefill_chunk_ranges.restype = I
-        L.dsa_prefill_chunk_ranges.argtypes = [P, P, P, I, P, P, I, I, I, I, I, P, P, I, F, I, P, P, P, P, Z, P]
+        L.dsa_prefill_chunk_ranges.argtypes = [P, P, LL, P, I, P, P, LL, I, I, I, I, I, P, P, I, F, I, P, P, P, P, Z,
+                                               P]
         L.dsa_selftest_wait_timeout.restype = I
         L.dsa_selftest_wait_timeout.argtypes = [P, Z, ctypes.c_uint, P]
         L.dsa_workspace_status.restype = I
@@ -95,6 +98,18 @@ def _dev(t: torch.Tensor | None, name: str, dtypes=None) -> int | None:
     if dtypes is not None and t.dtype not in dtypes:
         raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
     return t.data_ptr()
+
+
+def _rows(t: torch.Tensor, name: str, dtypes=None) -> tuple[int, int]:
+    """(pointer, row stride in elements) of a 2-D CUDA tensor whose rows are contiguous (a padded cache or
+    a view of the leading columns of a wider buffer)."""
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 2 or t.stride(1) != 1 or t.stride(0) < t.shape[1]:
+        raise ValueError(f"{name} must be 2-D with contiguous rows")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    return t.data_ptr(), t.stride(0)
 
 
 def _stream(stream) -> int | None:
@@ -153,7 +168,7 @@ def dsa_indexer_topk(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, 
     if workspace is None:
         workspace = alloc_workspace(dsa_indexer_topk_workspace(L, N, H_I, D_I, topk, dt), q_idx.device)
     _check(lib().dsa_indexer_topk(
-        _dev(q_idx, "q_idx"), _dev(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt, L, N, H_I, D_I, q_pos0,
+        _dev(q_idx, "q_idx"), *_rows(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt, L, N, H_I, D_I, q_pos0,
         topk, _dev(topk_idx, "topk_idx", (torch.int32,)), _dev(topk_score, "topk_score", (torch.float32,)),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)),
         "dsa_indexer_topk")
@@ -175,7 +190,7 @@ def dsa_indexer_topk_ranges(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.T
     if workspace is None:
         workspace = alloc_workspace(dsa_indexer_topk_workspace(L, N, H_I, D_I, topk, dt), q_idx.device)
     _check(lib().dsa_indexer_topk_ranges(
-        _dev(q_idx, "q_idx"), _dev(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt, L, N, H_I, D_I,
+        _dev(q_idx, "q_idx"), *_rows(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt, L, N, H_I, D_I,
         _dev(key_lo, "key_lo", (torch.int32,)), _dev(key_hi, "key_hi", (torch.int32,)), topk,
         _dev(topk_idx, "topk_idx", (torch.int32,)), _dev(topk_score, "topk_score", (torch.float32,)),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)),
@@ -197,7 +212,7 @@ def dsa_indexer_topk_noalloc(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.
     if tuple(topk_idx.shape) != (L, topk):
         raise ValueError("topk_idx must be [L, topk]")
     _check(lib().dsa_indexer_topk_noalloc(
-        _dev(q_idx, "q_idx"), _dev(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt, L, N, H_I, D_I, q_pos0,
+        _dev(q_idx, "q_idx"), *_rows(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt, L, N, H_I, D_I, q_pos0,
         topk, _dev(topk_idx, "topk_idx", (torch.int32,)), _dev(topk_score, "topk_score", (torch.float32,)),
         _stream(stream)), "dsa_indexer_topk_noalloc")
 
@@ -215,7 +230,7 @@ def dsa_sparse_mla_prefill(q: torch.Tensor, kv: torch.Tensor, topk_idx: torch.Te
     if workspace is None:
         workspace = alloc_workspace(dsa_sparse_mla_workspace(L, H, topk), q.device)
     _check(lib().dsa_sparse_mla_prefill(
-        _dev(q, "q", (torch.bfloat16,)), _dev(kv, "kv", (torch.bfloat16,)), _dev(topk_idx, "topk_idx", (torch.int32,)),
+        _dev(q, "q", (torch.bfloat16,)), *_rows(kv, "kv", (torch.bfloat16,)), _dev(topk_idx, "topk_idx", (torch.int32,)),
         L, N, H, topk, float(scale), _dev(out, "out", (torch.bfloat16,)), _dev(lse, "lse", (torch.float32,)),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)),
         "dsa_sparse_mla_prefill")
@@ -234,8 +249,8 @@ def dsa_prefill_chunk(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor,
         workspace = alloc_workspace(dsa_prefill_chunk_workspace(L, N, H_I, D_I, H, topk, query_block, dt,
                                                                 topk_idx is not None), q.device)
     _check(lib().dsa_prefill_chunk(
-        _dev(q_idx, "q_idx"), _dev(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt,
-        _dev(q, "q", (torch.bfloat16,)), _dev(kv, "kv", (torch.bfloat16,)), L, N, H_I, D_I, H, q_pos0, topk,
+        _dev(q_idx, "q_idx"), *_rows(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt,
+        _dev(q, "q", (torch.bfloat16,)), *_rows(kv, "kv", (torch.bfloat16,)), L, N, H_I, D_I, H, q_pos0, topk,
         float(scale), query_block, _dev(topk_idx, "topk_idx", (torch.int32,)), _dev(out, "out", (torch.bfloat16,)),
         _dev(lse, "lse", (torch.float32,)), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)), "dsa_prefill_chunk")
@@ -256,8 +271,8 @@ def dsa_prefill_chunk_ranges(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.
         workspace = alloc_workspace(dsa_prefill_chunk_workspace(L, N, H_I, D_I, H, topk, query_block, dt,
                                                                 topk_idx is not None), q.device)
     _check(lib().dsa_prefill_chunk_ranges(
-        _dev(q_idx, "q_idx"), _dev(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt,
-        _dev(q, "q", (torch.bfloat16,)), _dev(kv, "kv", (torch.bfloat16,)), L, N, H_I, D_I, H,
+        _dev(q_idx, "q_idx"), *_rows(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt,
+        _dev(q, "q", (torch.bfloat16,)), *_rows(kv, "kv", (torch.bfloat16,)), L, N, H_I, D_I, H,
         _dev(key_lo, "key_lo", (torch.int32,)), _dev(key_hi, "key_hi", (torch.int32,)), topk, float(scale),
         query_block, _dev(topk_idx, "topk_idx", (torch.int32,)), _dev(out, "out", (torch.bfloat16,)),
         _dev(lse, "lse", (torch.float32,)), _dev(workspace, "workspace"),
@@ -280,8 +295,8 @@ def dsa_prefill_chunk_profiled(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torc
                                                                 topk_idx is not None), q.device)
     handles = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     _check(lib().dsa_prefill_chunk_profiled(
-        _dev(q_idx, "q_idx"), _dev(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt,
-        _dev(q, "q", (torch.bfloat16,)), _dev(kv, "kv", (torch.bfloat16,)), L, N, H_I, D_I, H, q_pos0, topk,
+        _dev(q_idx, "q_idx"), *_rows(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt,
+        _dev(q, "q", (torch.bfloat16,)), *_rows(kv, "kv", (torch.bfloat16,)), L, N, H_I, D_I, H, q_pos0, topk,
         float(scale), query_block, _dev(topk_idx, "topk_idx", (torch.int32,)), _dev(out, "out", (torch.bfloat16,)),
         _dev(lse, "lse", (torch.float32,)), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream), handles, len(events)),

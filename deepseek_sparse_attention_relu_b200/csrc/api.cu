@@ -140,6 +140,8 @@ struct IndexerProblem {
   float *topk_score;
   // Per-query key ranges (device, [L]; nullptr = causal from q_pos0).
   const int32_t *key_lo = nullptr, *key_hi = nullptr;
+  long long ldk = 0;              // k_idx row stride in elements (0 = D_I, contiguous)
+  long long key_ld() const { return ldk > 0 ? ldk : D_I; }
 };
 
 dsa_status_t check_indexer_args(const IndexerProblem &p) {
@@ -157,6 +159,9 @@ dsa_status_t check_indexer_args(const IndexerProblem &p) {
   }
   if (p.topk > kMaxTopk) return DSA_ERR_UNSUPPORTED;
   if (!indexer_supported(p.D_I, p.H_I, p.fp8)) return DSA_ERR_UNSUPPORTED;
+  // k_idx rows may be padded: stride >= D_I, and every row 16-byte aligned (TMA)
+  if (p.ldk < 0 || (p.ldk > 0 && p.ldk < p.D_I)) return DSA_ERR_INVALID_ARG;
+  if ((p.key_ld() * (p.fp8 ? 1 : 2)) % 16 != 0) return DSA_ERR_INVALID_ARG;
   return DSA_OK;
 }
 
@@ -176,7 +181,7 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
   const int q_pos0 = p.q_pos0 + t0;
   const int sms = std::max(1, sm_count());
   const long long esz = p.fp8 ? 1 : 2;
-  const long long row_bytes = static_cast<long long>(p.D_I) * esz;
+  const long long row_bytes = p.key_ld() * esz;  // k_idx row pitch
 
   IndexerArgs ia{};
   ia.w = p.w + static_cast<long long>(t0) * p.H_I;
@@ -236,6 +241,7 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
   SelectArgs sa{};
   sa.q_idx = p.q_idx;
   sa.k_idx = p.k_idx;
+  sa.ldk = p.key_ld();
   sa.w = p.w;
   sa.dense = pilot ? ws.dense : nullptr;
   sa.tau = ws.tau;
@@ -297,7 +303,7 @@ bool make_indexer_maps(const IndexerProblem &p, CUtensorMap *tq, CUtensorMap *tk
   const uint32_t esz = p.fp8 ? 1 : 2;
   const uint64_t row_bytes = static_cast<uint64_t>(p.D_I) * esz;
   return make_map_2d(tq, p.q_idx, dt, p.D_I, static_cast<uint64_t>(p.L) * p.H_I, row_bytes, 128 / esz, 256) &&
-         make_map_2d(tk, p.k_idx, dt, p.D_I, p.N, row_bytes, 128 / esz, 128);
+         make_map_2d(tk, p.k_idx, dt, p.D_I, p.N, static_cast<uint64_t>(p.key_ld()) * esz, 128 / esz, 128);
 }
 
 struct MlaProblem {
@@ -307,6 +313,8 @@ struct MlaProblem {
   float scale;
   void *out;
   float *lse;
+  long long ldkv = 0;             // kv row stride in elements (0 = 576, contiguous)
+  long long kv_ld() const { return ldkv > 0 ? ldkv : 576; }
 };
 
 dsa_status_t check_mla_args(const MlaProblem &p) {
@@ -316,6 +324,8 @@ dsa_status_t check_mla_args(const MlaProblem &p) {
   if (p.lse != nullptr && !aligned16(p.lse)) return DSA_ERR_INVALID_ARG;
   if (p.L <= 0 || p.N <= 0 || p.H <= 0 || p.topk <= 0) return DSA_ERR_INVALID_ARG;
   if (!std::isfinite(p.scale)) return DSA_ERR_INVALID_ARG;
+  // kv rows may be padded: stride >= 576 elements, every row 16-byte aligned (16-byte copies)
+  if (p.ldkv < 0 || (p.ldkv > 0 && p.ldkv < 576) || (p.kv_ld() * 2) % 16 != 0) return DSA_ERR_INVALID_ARG;
   if (static_cast<long long>(p.L) * p.H >= (1ll << 31)) return DSA_ERR_UNSUPPORTED;
   return DSA_OK;
 }
@@ -388,6 +398,7 @@ dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, unsigned 
   MlaArgs a{};
   a.topk_idx = p.topk_idx;
   a.kv = p.kv;
+  a.kv_ld = p.kv_ld();
   a.out = static_cast<uint16_t *>(p.out);
   a.lse = p.lse;
   a.status = status;
@@ -486,14 +497,15 @@ size_t dsa_indexer_topk_workspace(int L, int N, int H_I, int D_I, int topk, dsa_
 
 namespace {
 
-dsa_status_t indexer_topk_impl(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype, int L,
-                               int N, int H_I, int D_I, int q_pos0, const int32_t *key_lo, const int32_t *key_hi,
-                               int topk, int32_t *topk_idx, float *topk_score, void *workspace,
+dsa_status_t indexer_topk_impl(const void *q_idx, const void *k_idx, int64_t ldk, const float *w, dsa_dtype_t dtype,
+                               int L, int N, int H_I, int D_I, int q_pos0, const int32_t *key_lo,
+                               const int32_t *key_hi, int topk, int32_t *topk_idx, float *topk_score, void *workspace,
                                size_t workspace_bytes, dsa_stream_t stream_) {
   if (dtype != DSA_BF16 && dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID_ARG;
   IndexerProblem p{q_idx, k_idx, w, dtype == DSA_FP8_E4M3, L, N, H_I, D_I, q_pos0, topk, topk_idx, topk_score};
   p.key_lo = key_lo;
   p.key_hi = key_hi;
+  p.ldk = ldk;
   dsa_status_t st = check_indexer_args(p);
   if (st != DSA_OK) return st;
   const int QB = std::min(L, kDefaultQueryBlock);
@@ -514,20 +526,20 @@ dsa_status_t indexer_topk_impl(const void *q_idx, const void *k_idx, const float
 
 extern "C" {
 
-dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype, int L,
-                              int N, int H_I, int D_I, int q_pos0, int topk, int32_t *topk_idx, float *topk_score,
-                              void *workspace, size_t workspace_bytes, dsa_stream_t stream) {
-  return indexer_topk_impl(q_idx, k_idx, w, dtype, L, N, H_I, D_I, q_pos0, nullptr, nullptr, topk, topk_idx,
+dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, int64_t ldk, const float *w, dsa_dtype_t dtype,
+                              int L, int N, int H_I, int D_I, int q_pos0, int topk, int32_t *topk_idx,
+                              float *topk_score, void *workspace, size_t workspace_bytes, dsa_stream_t stream) {
+  return indexer_topk_impl(q_idx, k_idx, ldk, w, dtype, L, N, H_I, D_I, q_pos0, nullptr, nullptr, topk, topk_idx,
                            topk_score, workspace, workspace_bytes, stream);
 }
 
-dsa_status_t dsa_indexer_topk_ranges(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
-                                     int L, int N, int H_I, int D_I, const int32_t *key_lo,
+dsa_status_t dsa_indexer_topk_ranges(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
+                                     dsa_dtype_t dtype, int L, int N, int H_I, int D_I, const int32_t *key_lo,
                                      const int32_t *key_hi, int topk, int32_t *topk_idx, float *topk_score,
                                      void *workspace, size_t workspace_bytes, dsa_stream_t stream) {
   if (key_lo == nullptr || key_hi == nullptr) return DSA_ERR_INVALID_ARG;
-  return indexer_topk_impl(q_idx, k_idx, w, dtype, L, N, H_I, D_I, 0, key_lo, key_hi, topk, topk_idx, topk_score,
-                           workspace, workspace_bytes, stream);
+  return indexer_topk_impl(q_idx, k_idx, ldk, w, dtype, L, N, H_I, D_I, 0, key_lo, key_hi, topk, topk_idx,
+                           topk_score, workspace, workspace_bytes, stream);
 }
 
 size_t dsa_sparse_mla_workspace(int L, int H, int topk) {
@@ -535,10 +547,11 @@ size_t dsa_sparse_mla_workspace(int L, int H, int topk) {
   return kHeaderBytes + attention_scratch_bytes(L, L, H, topk);
 }
 
-dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, const int32_t *topk_idx, int L, int N, int H,
-                                    int topk, float scale, void *out, float *lse, void *workspace,
+dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, int64_t ldkv, const int32_t *topk_idx, int L,
+                                    int N, int H, int topk, float scale, void *out, float *lse, void *workspace,
                                     size_t workspace_bytes, dsa_stream_t stream_) {
   MlaProblem p{q, kv, topk_idx, L, N, H, topk, scale, out, lse};
+  p.ldkv = ldkv;
   dsa_status_t st = check_mla_args(p);
   if (st != DSA_OK) return st;
   if (workspace == nullptr || workspace_bytes < kHeaderBytes) return DSA_ERR_WORKSPACE;
@@ -569,9 +582,9 @@ size_t dsa_prefill_chunk_workspace(int L, int N, int H_I, int D_I, int H, int to
 
 namespace {
 
-dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
-                                const void *q, const void *kv, int L, int N, int H_I, int D_I, int H, int q_pos0,
-                                const int32_t *key_lo, const int32_t *key_hi, int topk, float scale,
+dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, int64_t ldk, const float *w, dsa_dtype_t dtype,
+                                const void *q, const void *kv, int64_t ldkv, int L, int N, int H_I, int D_I, int H,
+                                int q_pos0, const int32_t *key_lo, const int32_t *key_hi, int topk, float scale,
                                 int query_block, int32_t *topk_idx_out, void *out, float *lse, void *workspace,
                                 size_t workspace_bytes, dsa_stream_t stream_, cudaEvent_t *events, int n_events) {
   if (dtype != DSA_BF16 && dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID_ARG;
@@ -600,9 +613,11 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, const floa
                     topk_idx_out ? topk_idx_out : block_idx, nullptr};
   ip.key_lo = key_lo;
   ip.key_hi = key_hi;
+  ip.ldk = ldk;
   dsa_status_t st = check_indexer_args(ip);
   if (st != DSA_OK) return st;
   MlaProblem mp{q, kv, ip.topk_idx, L, N, H, topk, scale, out, lse};
+  mp.ldkv = ldkv;
   st = check_mla_args(mp);
   if (st != DSA_OK) return st;
   IdxWorkspace ws;
@@ -636,32 +651,35 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, const floa
 
 extern "C" {
 
-dsa_status_t dsa_prefill_chunk(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
-                               const void *q, const void *kv, int L, int N, int H_I, int D_I, int H, int q_pos0,
-                               int topk, float scale, int query_block, int32_t *topk_idx_out, void *out, float *lse,
-                               void *workspace, size_t workspace_bytes, dsa_stream_t stream) {
-  return prefill_chunk_impl(q_idx, k_idx, w, dtype, q, kv, L, N, H_I, D_I, H, q_pos0, nullptr, nullptr, topk, scale,
-                            query_block, topk_idx_out, out, lse, workspace, workspace_bytes, stream, nullptr, 0);
+dsa_status_t dsa_prefill_chunk(const void *q_idx, const void *k_idx, int64_t ldk, const float *w, dsa_dtype_t dtype,
+                               const void *q, const void *kv, int64_t ldkv, int L, int N, int H_I, int D_I, int H,
+                               int q_pos0, int topk, float scale, int query_block, int32_t *topk_idx_out, void *out,
+                               float *lse, void *workspace, size_t workspace_bytes, dsa_stream_t stream) {
+  return prefill_chunk_impl(q_idx, k_idx, ldk, w, dtype, q, kv, ldkv, L, N, H_I, D_I, H, q_pos0, nullptr, nullptr,
+                            topk, scale, query_block, topk_idx_out, out, lse, workspace, workspace_bytes, stream,
+                            nullptr, 0);
 }
 
-dsa_status_t dsa_prefill_chunk_ranges(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
-                                      const void *q, const void *kv, int L, int N, int H_I, int D_I, int H,
-                                      const int32_t *key_lo, const int32_t *key_hi, int topk, float scale,
-                                      int query_block, int32_t *topk_idx_out, void *out, float *lse,
+dsa_status_t dsa_prefill_chunk_ranges(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
+                                      dsa_dtype_t dtype, const void *q, const void *kv, int64_t ldkv, int L, int N,
+                                      int H_I, int D_I, int H, const int32_t *key_lo, const int32_t *key_hi, int topk,
+                                      float scale, int query_block, int32_t *topk_idx_out, void *out, float *lse,
                                       void *workspace, size_t workspace_bytes, dsa_stream_t stream) {
   if (key_lo == nullptr || key_hi == nullptr) return DSA_ERR_INVALID_ARG;
-  return prefill_chunk_impl(q_idx, k_idx, w, dtype, q, kv, L, N, H_I, D_I, H, 0, key_lo, key_hi, topk, scale,
-                            query_block, topk_idx_out, out, lse, workspace, workspace_bytes, stream, nullptr, 0);
+  return prefill_chunk_impl(q_idx, k_idx, ldk, w, dtype, q, kv, ldkv, L, N, H_I, D_I, H, 0, key_lo, key_hi, topk,
+                            scale, query_block, topk_idx_out, out, lse, workspace, workspace_bytes, stream, nullptr,
+                            0);
 }
 
-dsa_status_t dsa_prefill_chunk_profiled(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
-                                        const void *q, const void *kv, int L, int N, int H_I, int D_I, int H,
-                                        int q_pos0, int topk, float scale, int query_block, int32_t *topk_idx_out,
-                                        void *out, float *lse, void *workspace, size_t workspace_bytes,
-                                        dsa_stream_t stream, void *const *events, int n_events) {
+dsa_status_t dsa_prefill_chunk_profiled(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
+                                        dsa_dtype_t dtype, const void *q, const void *kv, int64_t ldkv, int L, int N,
+                                        int H_I, int D_I, int H, int q_pos0, int topk, float scale, int query_block,
+                                        int32_t *topk_idx_out, void *out, float *lse, void *workspace,
+                                        size_t workspace_bytes, dsa_stream_t stream, void *const *events,
+                                        int n_events) {
   if (events == nullptr) return DSA_ERR_INVALID_ARG;
-  return prefill_chunk_impl(q_idx, k_idx, w, dtype, q, kv, L, N, H_I, D_I, H, q_pos0, nullptr, nullptr, topk, scale,
-                            query_block, topk_idx_out, out, lse, workspace, workspace_bytes, stream,
+  return prefill_chunk_impl(q_idx, k_idx, ldk, w, dtype, q, kv, ldkv, L, N, H_I, D_I, H, q_pos0, nullptr, nullptr,
+                            topk, scale, query_block, topk_idx_out, out, lse, workspace, workspace_bytes, stream,
                             reinterpret_cast<cudaEvent_t *>(const_cast<void **>(events)), n_events);
 }
 
@@ -727,12 +745,13 @@ dsa_status_t noalloc_scratch(void **out) {
 
 }  // namespace
 
-extern "C" dsa_status_t dsa_indexer_topk_noalloc(const void *q_idx, const void *k_idx, const float *w,
+extern "C" dsa_status_t dsa_indexer_topk_noalloc(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
                                                  dsa_dtype_t dtype, int L, int N, int H_I, int D_I, int q_pos0,
                                                  int topk, int32_t *topk_idx, float *topk_score,
                                                  dsa_stream_t stream_) {
   if (dtype != DSA_BF16 && dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID_ARG;
   IndexerProblem p{q_idx, k_idx, w, dtype == DSA_FP8_E4M3, L, N, H_I, D_I, q_pos0, topk, topk_idx, topk_score};
+  p.ldk = ldk;
   dsa_status_t st = check_indexer_args(p);
   if (st != DSA_OK) return st;
   const int QB = std::min(L, kNoAllocQueryBlock);

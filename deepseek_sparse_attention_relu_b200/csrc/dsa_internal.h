@@ -67,6 +67,7 @@ struct SelectArgs {
   int32_t *topk_idx;              // [L, topk] whole chunk
   float *topk_score;              // [L, topk] or nullptr
   int dense_ld, n_samples, cap, fb_slots;
+  long long ldk;                  // k_idx row stride in elements
   const int *key_lo, *key_hi;     // [Lb] clamped per-query ranges, or nullptr (causal)
   int sample_stride;              // with ranges: pilot sample i is key i * sample_stride
   int t0, Lb, q_pos0;             // block: first query (chunk row), size, position of first query
@@ -80,7 +81,8 @@ cudaError_t launch_fallback(const SelectArgs &a, cudaStream_t stream);
 // Sparse absorbed-MLA attention.
 struct MlaArgs {
   const int32_t *topk_idx;        // [L, topk]
-  const void *kv;                 // [N, 576] bf16 joined cache
+  const void *kv;                 // [N, 576] bf16 joined cache, rows kv_ld elements apart
+  long long kv_ld;
   uint16_t *out;                  // [L, H, 512] bf16 bits
   float *lse;                     // [L, H] or nullptr
   unsigned *status;

@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       return (PACKED && pw == 0 && lane < nq && j < ntiles) ? qmask[static_cast<long long>(j) * 64 + lane] : 0ull;
     };
     auto row_offset = [&](int v) -> long long {  // invalid entries read row 0 (their scores are masked)
-      return static_cast<long long>((v >= 0 && v < a.N) ? v : 0) * (DIM * 2);
+      return static_cast<long long>((v >= 0 && v < a.N) ? v : 0) * a.kv_ld * 2;
     };
     const uint8_t *kv = static_cast<const uint8_t *>(a.kv);
     // Index registers run one tile ahead.
@@ -235,14 +235,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < PPW; ++i) {
           const int r = 2 * (pw + N_PROD * i) + sub2;
           if (r < BK)
-            cp_async_16(stage_base + c * ATOM_BYTES + r * 128 + ((u ^ (r & 7)) << 4), kv + row_offset(kp[i]) + c * 128 + u * 16);
+            cp_async_16(stage_base + c * ATOM_BYTES + r * 128 + ((u ^ (r & 7)) << 4),
+                        kv + row_offset(kp[i]) + c * 128 + u * 16);
         }
       }
 #pragma unroll
       for (int i = 0; i < GPW; ++i) {
         const int r = 4 * (pw + N_PROD * i) + sub4;
         if (r < BK)
-          cp_async_16(stage_base + 8 * ATOM_BYTES + r * 128 + ((u ^ (r & 7)) << 4), kv + row_offset(kq[i]) + 8 * 128 + u * 16);
+          cp_async_16(stage_base + 8 * ATOM_BYTES + r * 128 + ((u ^ (r & 7)) << 4),
+                      kv + row_offset(kq[i]) + 8 * 128 + u * 16);
       }
       cp_async_arrive_noinc(&kv_full[st]);
       // Pull the next tile's rows from HBM into L2 now; its gather starts only

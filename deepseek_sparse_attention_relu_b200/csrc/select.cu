@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(SelectArgs a) {
     for (int j = threadIdx.x; j < nvis; j += blockDim.x) {
       const int s = lo + j;
       float kr[128];
-      for (int d = 0; d < a.D_I; ++d) kr[d] = idx_elem(a.k_idx, static_cast<long long>(s) * a.D_I + d, a.fp8);
+      for (int d = 0; d < a.D_I; ++d) kr[d] = idx_elem(a.k_idx, static_cast<long long>(s) * a.ldk + d, a.fp8);
       float score = 0.0f;
       for (int h = 0; h < a.H_I; ++h) {
         float dot = 0.0f;

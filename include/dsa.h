@@ -85,7 +85,11 @@ size_t dsa_indexer_topk_workspace(int L, int N, int H_I, int D_I, int topk, dsa_
  * Stages 1+2: lightning-indexer scores and exact top-k per query.
  *
  *   q_idx      [L, H_I, D_I]  indexer queries, dtype bits
- *   k_idx      [N, D_I]       indexer key cache, dtype bits
+ *   k_idx      [N, D_I]       indexer key cache, dtype bits; rows ldk elements
+ *                             apart (ldk = 0: D_I, contiguous; otherwise
+ *                             ldk >= D_I and every row 16-byte aligned, e.g. a
+ *                             padded cache or the leading columns of a wider
+ *                             buffer; the padding is never read)
  *   w          [L, H_I]       fp32 head weights (signed)
  *   topk_idx   [L, topk]      out: int32 selected keys, ascending, -1 padded
  *   topk_score [L, topk]      out (optional, may be NULL): fp32 indexer score
@@ -97,9 +101,10 @@ size_t dsa_indexer_topk_workspace(int L, int N, int H_I, int D_I, int topk, dsa_
  * up to 1,024 (mlx-lm PR #1997, "How it works": long chunks split into query
  * blocks); the result does not depend on the blocking.
  */
-dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype, int L,
-                              int N, int H_I, int D_I, int q_pos0, int topk, int32_t *topk_idx, float *topk_score,
-                              void *workspace, size_t workspace_bytes, dsa_stream_t stream);
+dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
+                              dsa_dtype_t dtype, int L, int N, int H_I, int D_I, int q_pos0, int topk,
+                              int32_t *topk_idx, float *topk_score, void *workspace, size_t workspace_bytes,
+                              dsa_stream_t stream);
 
 /*
  * dsa_indexer_topk for callers that cannot allocate device memory: code that
@@ -140,14 +145,14 @@ dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, const float 
  * another in the cache, query t of the sequence starting at key b sees
  * [b, its own position + 1).  Workspace: dsa_indexer_topk_workspace.
  */
-dsa_status_t dsa_indexer_topk_ranges(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
-                                     int L, int N, int H_I, int D_I, const int32_t *key_lo,
+dsa_status_t dsa_indexer_topk_ranges(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
+                                     dsa_dtype_t dtype, int L, int N, int H_I, int D_I, const int32_t *key_lo,
                                      const int32_t *key_hi, int topk, int32_t *topk_idx, float *topk_score,
                                      void *workspace, size_t workspace_bytes, dsa_stream_t stream);
 
-dsa_status_t dsa_indexer_topk_noalloc(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
-                                      int L, int N, int H_I, int D_I, int q_pos0, int topk, int32_t *topk_idx,
-                                      float *topk_score, dsa_stream_t stream);
+dsa_status_t dsa_indexer_topk_noalloc(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
+                                      dsa_dtype_t dtype, int L, int N, int H_I, int D_I, int q_pos0, int topk,
+                                      int32_t *topk_idx, float *topk_score, dsa_stream_t stream);
 
 /* Workspace (bytes) for dsa_sparse_mla_prefill: the status word, plus the
  * union buffers of packed attention (H <= 32) or the fp32 partial results of
@@ -161,7 +166,9 @@ size_t dsa_sparse_mla_workspace(int L, int H, int topk);
  * Stage 3: sparse absorbed-MLA attention.
  *
  *   q        [L, H, 576]  bf16: per head 512 latent then 64 rope columns
- *   kv       [N, 576]     bf16 joined cache: 512 latent then 64 rope columns
+ *   kv       [N, 576]     bf16 joined cache: 512 latent then 64 rope columns;
+ *                         rows ldkv elements apart (0: 576, contiguous;
+ *                         otherwise ldkv >= 576 with 16-byte aligned rows)
  *   topk_idx [L, topk]    int32 keys per query; -1 entries are skipped; any
  *                         order; values >= N are skipped and flagged
  *   out      [L, H, 512]  out: bf16 attention output
@@ -182,8 +189,8 @@ size_t dsa_sparse_mla_workspace(int L, int H, int topk);
  *     kernel).  The choice depends on L, H and topk only, never on a caller's
  *     query blocking.
  */
-dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, const int32_t *topk_idx, int L, int N, int H,
-                                    int topk, float scale, void *out, float *lse, void *workspace,
+dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, int64_t ldkv, const int32_t *topk_idx, int L,
+                                    int N, int H, int topk, float scale, void *out, float *lse, void *workspace,
                                     size_t workspace_bytes, dsa_stream_t stream);
 
 /* Workspace (bytes) for dsa_prefill_chunk with these sizes (query_block <= 0
@@ -195,28 +202,29 @@ size_t dsa_prefill_chunk_workspace(int L, int N, int H_I, int D_I, int H, int to
  * All three stages for one prefill chunk, query block by query block
  * (query_block <= 0 selects 1,024 queries per block).
  *
- *   q_idx, k_idx, w, dtype, H_I, D_I : as dsa_indexer_topk
- *   q, kv, H, scale                  : as dsa_sparse_mla_prefill
+ *   q_idx, k_idx, ldk, w, dtype, H_I, D_I : as dsa_indexer_topk
+ *   q, kv, ldkv, H, scale                 : as dsa_sparse_mla_prefill
  *   topk_idx_out [L, topk]           : optional (may be NULL) selected keys;
  *                                      when NULL they live in the workspace
  *   out [L, H, 512], lse [L, H]      : as dsa_sparse_mla_prefill (lse optional)
  *
  * want_topk_out of the workspace query must be 0 when topk_idx_out is NULL.
  */
-dsa_status_t dsa_prefill_chunk(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
-                               const void *q, const void *kv, int L, int N, int H_I, int D_I, int H, int q_pos0,
-                               int topk, float scale, int query_block, int32_t *topk_idx_out, void *out, float *lse,
-                               void *workspace, size_t workspace_bytes, dsa_stream_t stream);
+dsa_status_t dsa_prefill_chunk(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
+                               dsa_dtype_t dtype, const void *q, const void *kv, int64_t ldkv, int L, int N, int H_I,
+                               int D_I, int H, int q_pos0, int topk, float scale, int query_block,
+                               int32_t *topk_idx_out, void *out, float *lse, void *workspace, size_t workspace_bytes,
+                               dsa_stream_t stream);
 
 /*
  * dsa_prefill_chunk with general visibility: query t sees keys key_lo[t] <=
  * s < key_hi[t] (as dsa_indexer_topk_ranges) instead of the causal prefix
  * from q_pos0.  Workspace: dsa_prefill_chunk_workspace.
  */
-dsa_status_t dsa_prefill_chunk_ranges(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
-                                      const void *q, const void *kv, int L, int N, int H_I, int D_I, int H,
-                                      const int32_t *key_lo, const int32_t *key_hi, int topk, float scale,
-                                      int query_block, int32_t *topk_idx_out, void *out, float *lse,
+dsa_status_t dsa_prefill_chunk_ranges(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
+                                      dsa_dtype_t dtype, const void *q, const void *kv, int64_t ldkv, int L, int N,
+                                      int H_I, int D_I, int H, const int32_t *key_lo, const int32_t *key_hi, int topk,
+                                      float scale, int query_block, int32_t *topk_idx_out, void *out, float *lse,
                                       void *workspace, size_t workspace_bytes, dsa_stream_t stream);
 
 /*
@@ -227,11 +235,12 @@ dsa_status_t dsa_prefill_chunk_ranges(const void *q_idx, const void *k_idx, cons
  * after the threshold kernel, after the main indexer pass, after the
  * selection, after the exact fallback and after the attention kernel.
  */
-dsa_status_t dsa_prefill_chunk_profiled(const void *q_idx, const void *k_idx, const float *w, dsa_dtype_t dtype,
-                                        const void *q, const void *kv, int L, int N, int H_I, int D_I, int H,
-                                        int q_pos0, int topk, float scale, int query_block, int32_t *topk_idx_out,
-                                        void *out, float *lse, void *workspace, size_t workspace_bytes,
-                                        dsa_stream_t stream, void *const *events, int n_events);
+dsa_status_t dsa_prefill_chunk_profiled(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
+                                        dsa_dtype_t dtype, const void *q, const void *kv, int64_t ldkv, int L, int N,
+                                        int H_I, int D_I, int H, int q_pos0, int topk, float scale, int query_block,
+                                        int32_t *topk_idx_out, void *out, float *lse, void *workspace,
+                                        size_t workspace_bytes, dsa_stream_t stream, void *const *events,
+                                        int n_events);
 
 /*
  * Diagnostic with no counterpart in the method: exercises the bounded-wait

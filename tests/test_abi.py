@@ -58,7 +58,8 @@ def test_argument_errors_before_any_launch(lib):
     fake = 1 << 20  # a 16-byte-aligned non-null address that is never dereferenced
     ws = 1 << 24
     call = lambda **kw: lib.dsa_indexer_topk(  # noqa: E731
-        _P(kw.get("q", fake)), _P(kw.get("k", fake)), _P(kw.get("w", fake)), kw.get("dt", 0), kw.get("L", 4),
+        _P(kw.get("q", fake)), _P(kw.get("k", fake)), kw.get("ldk", 0), _P(kw.get("w", fake)), kw.get("dt", 0),
+        kw.get("L", 4),
         kw.get("N", 100), kw.get("H_I", 32), kw.get("D_I", 128), kw.get("q_pos0", 96), kw.get("topk", 8),
         _P(kw.get("idx", fake)), None, _P(ws), 1 << 30, None)
     assert call(q=0) == 1                 # null pointer
@@ -71,11 +72,17 @@ def test_argument_errors_before_any_launch(lib):
     assert call(topk=5000) == 2           # beyond the supported top-k
     assert call(H_I=3) == 2               # unsupported head count
     assert call(D_I=96) == 2
-    st = lib.dsa_sparse_mla_prefill(_P(fake), _P(fake), _P(0), 4, 100, 8, 16, ctypes.c_float(0.1), _P(fake), None,
-                                    _P(ws), 256, None)
+    assert call(ldk=100) == 1             # row stride shorter than a row
+    assert call(ldk=132) == 1             # rows not 16-byte aligned (132 bf16 = 264 B)
+    assert call(ldk=136) != 1             # a padded, aligned stride is accepted by the checks
+    st = lib.dsa_sparse_mla_prefill(_P(fake), _P(fake), 0, _P(0), 4, 100, 8, 16, ctypes.c_float(0.1), _P(fake),
+                                    None, _P(ws), 256, None)
     assert st == 1
-    st = lib.dsa_sparse_mla_prefill(_P(fake), _P(fake), _P(fake), 4, 100, 8, 16, ctypes.c_float(0.1), _P(fake), None,
-                                    None, 0, None)
+    st = lib.dsa_sparse_mla_prefill(_P(fake), _P(fake), 580, _P(fake), 4, 100, 8, 16, ctypes.c_float(0.1),
+                                    _P(fake), None, _P(ws), 256, None)
+    assert st == 1                        # kv rows not 16-byte aligned
+    st = lib.dsa_sparse_mla_prefill(_P(fake), _P(fake), 0, _P(fake), 4, 100, 8, 16, ctypes.c_float(0.1), _P(fake),
+                                    None, None, 0, None)
     assert st == 3                        # no workspace
 
 
