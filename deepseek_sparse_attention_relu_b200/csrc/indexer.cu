@@ -17,11 +17,17 @@
 //
 // Tile shape (swap-AB): A = 128 keys x D_I (UMMA M = 128), B = a group of
 // 256 / H_I queries x H_I heads = 256 rows x D_I (UMMA N = 256), K = D_I.
-// Each TMEM lane then holds one key and each epilogue thread reduces the heads
-// of its key locally.  Warp roles: warp 0 TMA producer, warp 1 MMA issuer and
-// TMEM owner, warps 2..17 epilogue (four per TMEM lane quarter, each taking 64
-// of the 256 accumulator columns).  The accumulator is double-buffered
-// (2 x 256 columns) so the epilogue of tile i overlaps the MMA of tile i+1.
+// Each TMEM lane then holds one key.  Warp roles: warp 0 TMA producer, warp 1
+// MMA issuer and TMEM owner, warps 2..17 epilogue (four per TMEM lane quarter,
+// each taking 64 of the 256 accumulator columns).  The accumulator is
+// double-buffered (2 x 256 columns) so the epilogue of tile i overlaps the MMA
+// of tile i+1.  With H_I a multiple of 8 the epilogue reads the accumulator in
+// 16-lane x 256-bit pieces: a thread then sees four keys but only a quarter of
+// the heads, so its head weights (16 values) stay in registers for the whole
+// query group instead of being re-read from shared memory every tile (per-lane
+// shared loads of the weights had kept the load/store unit's register
+// write-back busy 60% of the time), and four partial sums per score are added
+// across the thread quad with two shuffles.
 #include <cuda_runtime.h>
 
 #include "dsa_internal.h"
@@ -83,6 +89,10 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   z.f = c;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.u) : "l"(x.u), "l"(y.u), "l"(z.u));
   return r.f;
+}
+
+__device__ __forceinline__ float2 relu2(uint32_t a, uint32_t b) {
+  return make_float2(fmaxf(__uint_as_float(a), 0.0f), fmaxf(__uint_as_float(b), 0.0f));
 }
 
 // Threshold key -> float: a score s passes iff s >= threshold_float(key).  Key 0
@@ -338,6 +348,11 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     static_assert(3 * C::QH <= C::COLS, "thresholds and ranges share the per-warp slot");
     unsigned long long *stg = reinterpret_cast<unsigned long long *>(smem + C::OFF_STG) + ew * QH * SB;
     int cnt[QH];                   // staged candidates per query (warp-uniform)
+    // Indexer heads in whole 8-column blocks: 16-lane accumulator loads with the
+    // warp's head weights held in registers for the whole query group.
+    constexpr bool QUAD = (HI % 8) == 0;
+    const int c4 = lane & 3, r4 = lane >> 2;
+    float2 wreg[QH][HI / 8 > 0 ? HI / 8 : 1];
 #pragma unroll
     for (int qq = 0; qq < QH; ++qq) cnt[qq] = 0;
 
@@ -368,9 +383,21 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
         // Each warp stages the head weights / thresholds of its own queries
         // (no cross-warp barrier, so an aborting warp cannot strand the others).
         __syncwarp();
-        for (int j = lane; j < C::COLS; j += 32) {
-          const int tl = g * C::QG + slot * QH + j / HI;
-          w_w[j] = (tl < a.Lb) ? a.w[static_cast<long long>(g * C::QG + slot * QH) * HI + j] : 0.0f;
+        if constexpr (QUAD) {
+#pragma unroll
+          for (int qq = 0; qq < QH; ++qq) {
+            const int tl = g * C::QG + slot * QH + qq;
+#pragma unroll
+            for (int hp = 0; hp < HI / 8; ++hp) {
+              const long long o = static_cast<long long>(tl) * HI + 8 * hp + 2 * c4;
+              wreg[qq][hp] = (tl < a.Lb) ? make_float2(a.w[o], a.w[o + 1]) : make_float2(0.0f, 0.0f);
+            }
+          }
+        } else {
+          for (int j = lane; j < C::COLS; j += 32) {
+            const int tl = g * C::QG + slot * QH + j / HI;
+            w_w[j] = (tl < a.Lb) ? a.w[static_cast<long long>(g * C::QG + slot * QH) * HI + j] : 0.0f;
+          }
         }
         if (!PILOT) {
           for (int j = lane; j < QH; j += 32) {
@@ -389,37 +416,10 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
       tc_fence_after();
       const unsigned taddr =
           tmem_base + (static_cast<unsigned>(quarter * 32) << 16) + acc * 256 + slot * C::COLS;
-      const int key = c.key0() + quarter * 32 + lane;
-      // One 32-column chunk of the accumulator at a time (keeps the live
-      // register set small); the buffer goes back to the MMA warp after the
-      // last chunk has been read.
-#pragma unroll
-      for (int ch = 0; ch < C::COLS / 32; ++ch) {
-      uint32_t vc[32];
-      tmem_ld_32x32b_x32(taddr + ch * 32, vc);
-      tmem_ld_wait();
-      if (ch == C::COLS / 32 - 1) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      }
-#pragma unroll
-      for (int qq = ch * 32 / HI; qq < (ch + 1) * 32 / HI; ++qq) {
+      // Score of (query qq of this warp, key): dense write (pilot) or threshold
+      // test and staging (main pass).  Called by all 32 lanes together.
+      auto emit = [&](int qq, int key, float score) {
         const int tl = g * C::QG + slot * QH + qq;  // query within the block
-        const float4 *wq = reinterpret_cast<const float4 *>(w_w + qq * HI);
-        float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int h4 = 0; h4 < HI / 4; ++h4) {
-          const float4 w4 = wq[h4];
-          const int col = qq * HI + 4 * h4;
-          const float r0 = fmaxf(__uint_as_float(vc[(col + 0) % 32]), 0.0f);
-          const float r1 = fmaxf(__uint_as_float(vc[(col + 1) % 32]), 0.0f);
-          const float r2 = fmaxf(__uint_as_float(vc[(col + 2) % 32]), 0.0f);
-          const float r3 = fmaxf(__uint_as_float(vc[(col + 3) % 32]), 0.0f);
-          acc0 = ffma2(make_float2(w4.x, w4.y), make_float2(r0, r1), acc0);
-          acc1 = ffma2(make_float2(w4.z, w4.w), make_float2(r2, r3), acc1);
-        }
-        const float score = (acc0.x + acc1.x) + (acc0.y + acc1.y);
         if (PILOT) {
           if (tl < a.Lb && key < a.n_keys) a.dense[static_cast<long long>(tl) * a.dense_ld + key] = score;
         } else {
@@ -437,7 +437,88 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
             cnt[qq] += n;
           }
         }
-      }
+      };
+      if constexpr (QUAD) {
+        // 16-lane loads: this thread sees keys r4, r4 + 8, r4 + 16, r4 + 24 of the
+        // warp's 32 and, in every 8-column block, the two heads 2*c4, 2*c4 + 1.
+        // Its partial sums over those heads are added across the four threads
+        // of its quad; the thread ends with key r4 + 8*c4 for every query.
+        const int key = c.key0() + quarter * 32 + r4 + 8 * c4;
+        constexpr int NQ = 32 / HI;  // queries per 32-column chunk
+#pragma unroll
+        for (int ch = 0; ch < C::COLS / 32; ++ch) {
+          uint32_t va[16], vb[16];
+          tmem_ld_16x256b_x4(taddr + ch * 32, va);
+          tmem_ld_16x256b_x4(taddr + (16u << 16) + ch * 32, vb);
+          tmem_ld_wait();
+          if (ch == C::COLS / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          }
+          float2 pa[NQ][4];
+#pragma unroll
+          for (int qc = 0; qc < NQ; ++qc)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) pa[qc][kk] = make_float2(0.0f, 0.0f);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int qc = (8 * j) / HI;
+            const float2 wv = wreg[ch * NQ + qc][((8 * j) % HI) / 8];
+            pa[qc][0] = ffma2(wv, relu2(va[4 * j], va[4 * j + 1]), pa[qc][0]);
+            pa[qc][1] = ffma2(wv, relu2(va[4 * j + 2], va[4 * j + 3]), pa[qc][1]);
+            pa[qc][2] = ffma2(wv, relu2(vb[4 * j], vb[4 * j + 1]), pa[qc][2]);
+            pa[qc][3] = ffma2(wv, relu2(vb[4 * j + 2], vb[4 * j + 3]), pa[qc][3]);
+          }
+#pragma unroll
+          for (int qc = 0; qc < NQ; ++qc) {
+            // Reduce-scatter over the quad: lane bit 1 picks keys {0,1} or {2,3},
+            // lane bit 0 one of the pair.  Every thread adds the same four
+            // partials in the same tree, ((p0 + p2) + (p1 + p3)).
+            const float v0 = pa[qc][0].x + pa[qc][0].y, v1 = pa[qc][1].x + pa[qc][1].y;
+            const float v2 = pa[qc][2].x + pa[qc][2].y, v3 = pa[qc][3].x + pa[qc][3].y;
+            const bool b1 = (c4 & 2) != 0, b0 = (c4 & 1) != 0;
+            float k0 = b1 ? v2 : v0, k1 = b1 ? v3 : v1;
+            k0 += __shfl_xor_sync(0xffffffffu, b1 ? v0 : v2, 2);
+            k1 += __shfl_xor_sync(0xffffffffu, b1 ? v1 : v3, 2);
+            float score = b0 ? k1 : k0;
+            score += __shfl_xor_sync(0xffffffffu, b0 ? k0 : k1, 1);
+            emit(ch * NQ + qc, key, score);
+          }
+        }
+      } else {
+        const int key = c.key0() + quarter * 32 + lane;
+        // One 32-column chunk of the accumulator at a time (keeps the live
+        // register set small); the buffer goes back to the MMA warp after the
+        // last chunk has been read.
+#pragma unroll
+        for (int ch = 0; ch < C::COLS / 32; ++ch) {
+          uint32_t vc[32];
+          tmem_ld_32x32b_x32(taddr + ch * 32, vc);
+          tmem_ld_wait();
+          if (ch == C::COLS / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          }
+#pragma unroll
+          for (int qq = ch * 32 / HI; qq < (ch + 1) * 32 / HI; ++qq) {
+            const float4 *wq = reinterpret_cast<const float4 *>(w_w + qq * HI);
+            float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int h4 = 0; h4 < HI / 4; ++h4) {
+              const float4 w4 = wq[h4];
+              const int col = qq * HI + 4 * h4;
+              const float r0 = fmaxf(__uint_as_float(vc[(col + 0) % 32]), 0.0f);
+              const float r1 = fmaxf(__uint_as_float(vc[(col + 1) % 32]), 0.0f);
+              const float r2 = fmaxf(__uint_as_float(vc[(col + 2) % 32]), 0.0f);
+              const float r3 = fmaxf(__uint_as_float(vc[(col + 3) % 32]), 0.0f);
+              acc0 = ffma2(make_float2(w4.x, w4.y), make_float2(r0, r1), acc0);
+              acc1 = ffma2(make_float2(w4.z, w4.w), make_float2(r2, r3), acc1);
+            }
+            emit(qq, key, (acc0.x + acc1.x) + (acc0.y + acc1.y));
+          }
+        }
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       idx_cursor_next<RANGES>(c, a, C::QG);

@@ -226,6 +226,18 @@ __device__ __forceinline__ void tmem_ld_16x32bx2_x32(unsigned taddr, uint32_t (&
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+// 16 lanes x 256 bit, four repeats along the columns (32 columns in all).  For
+// repeat j, thread t gets r[4j], r[4j+1] = lane base + t/4, columns
+// col + 8j + 2(t%4) + {0, 1}, and r[4j+2], r[4j+3] = lane base + 8 + t/4, the
+// same two columns.
+__device__ __forceinline__ void tmem_ld_16x256b_x4(unsigned taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
