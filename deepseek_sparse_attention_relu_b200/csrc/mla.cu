@@ -532,17 +532,28 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(MlaArgs a) {
   float acc[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
-  for (int sp = 0; sp < a.nsplit; ++sp) {
-    const float ws = __shfl_sync(0xffffffffu, wgt, sp) * inv;
-    if (ws == 0.0f) continue;
-    const float4 *src = reinterpret_cast<const float4 *>(a.part_o + (rowg * a.nsplit + sp) * LAT + lane * 16);
+  // Four shares' loads in flight at a time (the shares are added in order;
+  // an empty share has weight 0 and its row, which may hold anything, is skipped).
+  for (int sp0 = 0; sp0 < a.nsplit; sp0 += 4) {
+    float4 v[4][4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float4 v = src[e];
-      acc[4 * e] += ws * v.x;
-      acc[4 * e + 1] += ws * v.y;
-      acc[4 * e + 2] += ws * v.z;
-      acc[4 * e + 3] += ws * v.w;
+    for (int j = 0; j < 4; ++j) {
+      const int sp = min(sp0 + j, a.nsplit - 1);
+      const float4 *src = reinterpret_cast<const float4 *>(a.part_o + (rowg * a.nsplit + sp) * LAT + lane * 16);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[j][e] = src[e];
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float ws = __shfl_sync(0xffffffffu, wgt, sp0 + j) * inv;  // lanes >= nsplit carry weight 0
+      if (sp0 + j >= a.nsplit || ws == 0.0f) continue;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[4 * e] += ws * v[j][e].x;
+        acc[4 * e + 1] += ws * v[j][e].y;
+        acc[4 * e + 2] += ws * v[j][e].z;
+        acc[4 * e + 3] += ws * v[j][e].w;
+      }
     }
   }
   const long long orow = (static_cast<long long>(a.t0) * a.H + rowg) * LAT + lane * 16;
