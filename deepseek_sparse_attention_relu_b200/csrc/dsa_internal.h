@@ -8,6 +8,29 @@
 
 namespace dsa {
 
+// Launch a kernel of this library on `stream` with programmatic stream
+// serialisation: the grid may be scheduled while the previous kernel in the
+// stream is still running.  Every kernel of the library starts with
+// pdl_wait_and_release() (ptx.cuh), which blocks until all prerequisite grids
+// have completed and their memory is visible, so the ordering seen by the
+// kernel's code is exactly that of a plain launch; only the launch latency
+// overlaps the predecessor's tail.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                 Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Arguments of one indexer launch (one query block).
 struct IndexerArgs {
   const float *w;                 // [Lb, H_I] head weights of the block's queries

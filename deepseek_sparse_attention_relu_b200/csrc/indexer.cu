@@ -180,6 +180,7 @@ template <int DI, int HI, bool FP8, bool PILOT, bool RANGES>
 __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    IndexerArgs a) {
+  pdl_wait_and_release();
   using C = IdxCfg<DI, HI, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -548,8 +549,7 @@ static cudaError_t launch_indexer_t(const CUtensorMap &tq, const CUtensorMap &tk
   auto kern = indexer_kernel<DI, HI, FP8, PILOT, RANGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, a);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream, tq, tk, a);
 }
 
 int indexer_queries_per_group(int H_I) { return 256 / H_I; }

@@ -80,6 +80,7 @@ __device__ __forceinline__ float fast_exp2(float x) {
 template <bool PACKED>
 __global__ void __launch_bounds__(THREADS, 1)
     sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q, MlaArgs a) {
+  pdl_wait_and_release();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *q_s = smem + OFF_Q;
@@ -515,6 +516,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 // lse = log sum_s exp(lse_s) and out = sum_s exp(lse_s - lse) o_s, which is
 // the softmax over the union of the shares (they are disjoint).
 __global__ void __launch_bounds__(256) mla_combine_kernel(MlaArgs a) {
+  pdl_wait_and_release();
   const int lane = threadIdx.x % 32;
   const long long rowg = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
   if (rowg >= static_cast<long long>(a.Lq) * a.H) return;
@@ -575,8 +577,7 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(MlaArgs a) {
 cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t stream) {
   const long long rows = static_cast<long long>(a.Lq) * a.H;
   const int blocks = static_cast<int>((rows * 32 + 255) / 256);
-  mla::mla_combine_kernel<<<blocks, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(mla::mla_combine_kernel, dim3(blocks), dim3(256), 0, stream, a);
 }
 
 cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, bool packed, cudaStream_t stream) {
@@ -585,8 +586,7 @@ cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, bool pack
   if (e != cudaSuccess) return e;
   dim3 grid(packed ? (a.Lq + a.G - 1) / a.G : a.Lq, packed ? 1 : (a.H + mla::HT - 1) / mla::HT,
             packed ? 1 : max(1, a.nsplit));
-  kern<<<grid, mla::THREADS, mla::SMEM_BYTES, stream>>>(tq, a);
-  return cudaGetLastError();
+  return launch_kernel(kern, grid, dim3(mla::THREADS), mla::SMEM_BYTES, stream, tq, a);
 }
 
 }  // namespace dsa

@@ -16,6 +16,15 @@ enum : unsigned {
   DEV_FALLBACK_FULL = 1u << 3 // more fallback queries than fallback capacity
 };
 
+// First statement of every kernel of the library: wait until the grids this
+// one depends on (the previous kernel in the stream) have completed and their
+// memory operations are visible -- a no-op for a plain launch -- then allow
+// the next kernel in the stream to be scheduled.
+__device__ __forceinline__ void pdl_wait_and_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Wall-clock budget of one wait, in nanoseconds (%globaltimer).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 

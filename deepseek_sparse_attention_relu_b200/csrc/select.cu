@@ -91,6 +91,7 @@ __device__ void block_radix_select(Fetch fetch, int n, int need, KeyT &prefix_ou
 constexpr int kMaxSamples = 4096;
 
 __global__ void __launch_bounds__(256) threshold_kernel(SelectArgs a) {
+  pdl_wait_and_release();
   __shared__ unsigned hist[256];
   __shared__ unsigned misc[4];
   __shared__ unsigned keys[kMaxSamples];  // the query's sample scores as order-preserving keys
@@ -182,6 +183,7 @@ __device__ int block_exclusive_scan(int v, int *warp_tot, int *total) {
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
+  pdl_wait_and_release();
   extern __shared__ __align__(16) unsigned char sel_smem[];
   unsigned long long *cs = reinterpret_cast<unsigned long long *>(sel_smem);         // staged candidates
   unsigned char *region = sel_smem + static_cast<size_t>(min(a.cap, kSmemCand)) * 8;  // bitmap or sort buffer
@@ -290,6 +292,7 @@ __device__ __forceinline__ float idx_elem(const void *base, long long i, int fp8
 }
 
 __global__ void __launch_bounds__(kSelThreads) fallback_kernel(SelectArgs a) {
+  pdl_wait_and_release();
   extern __shared__ float fb_smem[];
   __shared__ unsigned hist[256];
   __shared__ unsigned misc[4];
@@ -378,6 +381,7 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(SelectArgs a) {
 // waits on an mbarrier that nothing arrives on, gives up after limit_ns and
 // records DEV_TIMEOUT, exactly as a kernel whose producer stalled would.
 __global__ void wait_timeout_probe_kernel(unsigned *status, unsigned long long limit_ns) {
+  pdl_wait_and_release();
   __shared__ uint64_t never;
   if (threadIdx.x != 0) return;
   mbar_init(&never, 1);
@@ -386,8 +390,7 @@ __global__ void wait_timeout_probe_kernel(unsigned *status, unsigned long long l
 }
 
 cudaError_t launch_wait_timeout_probe(unsigned *status, unsigned long long limit_ns, cudaStream_t stream) {
-  wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
-  return cudaGetLastError();
+  return launch_kernel(wait_timeout_probe_kernel, dim3(1), dim3(32), 0, stream, status, limit_ns);
 }
 
 // ------------------------------------------------------------------ range plan
@@ -396,6 +399,7 @@ cudaError_t launch_wait_timeout_probe(unsigned *status, unsigned long long limit
 // window of 128-key tiles that covers its queries' non-empty ranges, and the
 // exclusive prefix of the windows' sizes for the indexer's work split.
 __global__ void __launch_bounds__(128) range_plan_kernel(RangePlanArgs a) {
+  pdl_wait_and_release();
   __shared__ int cnt_s[128];
   const int G = (a.Lb + a.QG - 1) / a.QG;
   for (int t = threadIdx.x; t < a.Lb; t += blockDim.x) {
@@ -438,8 +442,7 @@ __global__ void __launch_bounds__(128) range_plan_kernel(RangePlanArgs a) {
 
 cudaError_t launch_range_plan(const RangePlanArgs &a, cudaStream_t stream) {
   if ((a.Lb + a.QG - 1) / a.QG > 128) return cudaErrorInvalidValue;
-  range_plan_kernel<<<1, 128, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(range_plan_kernel, dim3(1), dim3(128), 0, stream, a);
 }
 
 // ------------------------------------------------------------------ pack plan
@@ -454,6 +457,7 @@ cudaError_t launch_range_plan(const RangePlanArgs &a, cudaStream_t stream) {
 constexpr int kPackThreads = 1024;
 
 __global__ void __launch_bounds__(kPackThreads) pack_plan_kernel(PackArgs a) {
+  pdl_wait_and_release();
   extern __shared__ unsigned pk_words[];  // bitmap [nwords], then exclusive prefix counts [nwords]
   __shared__ int warp_tot[kPackThreads / 32];
   __shared__ int total, nvalid_s, bad_s;
@@ -542,13 +546,11 @@ cudaError_t launch_pack_plan(const PackArgs &a, cudaStream_t stream) {
   if (smem > 200 * 1024 || a.G > 64) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(pack_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  pack_plan_kernel<<<npacks, kPackThreads, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(pack_plan_kernel, dim3(npacks), dim3(kPackThreads), smem, stream, a);
 }
 
 cudaError_t launch_threshold(const SelectArgs &a, cudaStream_t stream) {
-  threshold_kernel<<<a.Lb, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(threshold_kernel, dim3(a.Lb), dim3(256), 0, stream, a);
 }
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream) {
@@ -556,14 +558,12 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream) {
   const int smem = min(a.cap, kSmemCand) * 8 + max(kBitmapKeys / 8, kMaxTopk * 8);
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  select_kernel<<<a.Lb, kSelThreads, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(select_kernel, dim3(a.Lb), dim3(kSelThreads), smem, stream, a);
 }
 
 cudaError_t launch_fallback(const SelectArgs &a, cudaStream_t stream) {
   const int smem = (a.H_I * a.D_I + a.H_I) * static_cast<int>(sizeof(float));
-  fallback_kernel<<<a.fb_slots, kSelThreads, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(fallback_kernel, dim3(a.fb_slots), dim3(kSelThreads), smem, stream, a);
 }
 
 }  // namespace dsa
