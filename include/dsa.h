@@ -25,15 +25,21 @@
  * Conventions for every entry point
  *   - Query t of a chunk sits at position q_pos0 + t and sees keys 0..q_pos0+t
  *     (inclusive causality, position == key index).  0 <= q_pos0, q_pos0+L <= N.
- *   - All tensor arguments are DEVICE pointers to contiguous row-major
- *     buffers owned by the caller; the library allocates no device memory and
- *     keeps no state between calls.  Pointers must be 16-byte aligned.
+ *   - All tensor arguments are DEVICE pointers to row-major buffers owned by
+ *     the caller, contiguous except for the row strides of the key caches
+ *     (ldk, ldkv); the library allocates no device memory and keeps no state
+ *     between calls (dsa_indexer_topk_noalloc's fixed scratch aside).
+ *     Pointers must be 16-byte aligned.
  *   - bf16 / fp8 buffers are passed as raw bits (uint16 / uint8 storage).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
- *     default stream).  Argument errors are returned before anything is
- *     launched; a failed launch returns DSA_ERR_CUDA.  Device-side conditions
- *     (a wait that timed out, an out-of-range index) are recorded in the
- *     workspace's status word and read back with dsa_workspace_status().
+ *     default stream) and keep its order with the caller's other work.  The
+ *     library's own kernels use programmatic dependent launch: each may be
+ *     scheduled while its predecessor in the stream finishes, but waits for
+ *     that predecessor to complete before it touches memory.  Argument errors
+ *     are returned before anything is launched; a failed launch returns
+ *     DSA_ERR_CUDA.  Device-side conditions (a wait that timed out, an
+ *     out-of-range index) are recorded in the workspace's status word and read
+ *     back with dsa_workspace_status().
  *   - No function aborts the process or throws across the ABI.
  */
 #ifndef DSA_H_
