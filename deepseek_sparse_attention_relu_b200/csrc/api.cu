@@ -344,7 +344,7 @@ constexpr float kMaxUnionRatio = 0.75f; // pack when the union is at most 75% of
 // adds tensor work (the rows were idle) while shared keys are gathered once.
 // Capped so the attention grid still covers the GPU at least twice.
 int pack_group(int H, int topk, int Lq, int N) {
-  if (H > 32 || N > 800 * 1024) return 1;  // the pack plan's key bitmap must fit in shared memory
+  if (H <= 0 || topk <= 0 || H > 32 || N > 800 * 1024) return 1;  // the pack plan's key bitmap must fit in shared memory
   int G = std::min(64 / H, 8);  // the attention kernel tracks up to 8 queries per CTA
   G = std::min(G, kPackMaxEntries / topk);
   G = std::min(G, std::max(1, Lq / (2 * std::max(1, sm_count()))));
@@ -366,7 +366,7 @@ size_t union_bytes(int Lq, int topk) {
 int mla_splits(int L, int H, int topk) {
   const int items = L * ((H + 63) / 64);
   const int sms = std::max(1, sm_count());
-  if (2 * items > sms) return 1;
+  if (items <= 0 || 2 * items > sms) return 1;
   return std::max(1, std::min({16, (topk + 127) / 128, sms / items}));
 }
 
@@ -588,7 +588,8 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, int64_t ld
                                 int query_block, int32_t *topk_idx_out, void *out, float *lse, void *workspace,
                                 size_t workspace_bytes, dsa_stream_t stream_, cudaEvent_t *events, int n_events) {
   if (dtype != DSA_BF16 && dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID_ARG;
-  if (L <= 0 || topk <= 0) return DSA_ERR_INVALID_ARG;
+  // Sizes first: the scratch planning below divides by them.
+  if (L <= 0 || N <= 0 || H_I <= 0 || D_I <= 0 || H <= 0 || topk <= 0) return DSA_ERR_INVALID_ARG;
   const int QB = std::min(L, query_block > 0 ? query_block : kDefaultQueryBlock);
   // Selected keys: the caller's buffer, or a block-sized region at the end of the workspace.
   size_t idx_bytes = workspace_bytes;

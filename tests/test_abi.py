@@ -54,7 +54,11 @@ def _P(x):
 
 
 def test_argument_errors_before_any_launch(lib):
-    """Shape / pointer errors come back synchronously; no CUDA call is made (this runs without a GPU)."""
+    """Shape / pointer errors come back synchronously, before any launch or copy.
+
+    Every call here fails a host-side check, so the fake pointers are never
+    handed to the device (valid strides are exercised with real buffers by
+    the GPU tests)."""
     fake = 1 << 20  # a 16-byte-aligned non-null address that is never dereferenced
     ws = 1 << 24
     call = lambda **kw: lib.dsa_indexer_topk(  # noqa: E731
@@ -74,7 +78,6 @@ def test_argument_errors_before_any_launch(lib):
     assert call(D_I=96) == 2
     assert call(ldk=100) == 1             # row stride shorter than a row
     assert call(ldk=132) == 1             # rows not 16-byte aligned (132 bf16 = 264 B)
-    assert call(ldk=136) != 1             # a padded, aligned stride is accepted by the checks
     st = lib.dsa_sparse_mla_prefill(_P(fake), _P(fake), 0, _P(0), 4, 100, 8, 16, ctypes.c_float(0.1), _P(fake),
                                     None, _P(ws), 256, None)
     assert st == 1
@@ -84,6 +87,35 @@ def test_argument_errors_before_any_launch(lib):
     st = lib.dsa_sparse_mla_prefill(_P(fake), _P(fake), 0, _P(fake), 4, 100, 8, 16, ctypes.c_float(0.1), _P(fake),
                                     None, None, 0, None)
     assert st == 3                        # no workspace
+
+
+def test_argument_errors_other_entry_points(lib):
+    """The chunk, per-query-range, profiled and self-test entry points also refuse bad arguments up front."""
+    fake = 1 << 20
+    ws = 1 << 24
+    scale = ctypes.c_float(0.1)
+    # per-query key ranges without the range arrays
+    assert lib.dsa_indexer_topk_ranges(_P(fake), _P(fake), 0, _P(fake), 0, 4, 100, 32, 128, None, None, 8,
+                                       _P(fake), None, _P(ws), 1 << 30, None) == 1
+    assert lib.dsa_prefill_chunk_ranges(_P(fake), _P(fake), 0, _P(fake), 0, _P(fake), _P(fake), 0, 4, 100, 32, 128,
+                                        64, None, None, 8, scale, 0, _P(fake), _P(fake), None, _P(ws), 1 << 30,
+                                        None) == 1
+
+    def chunk(dt=0, ldkv=0, q_pos0=96, H=64):
+        return lib.dsa_prefill_chunk(_P(fake), _P(fake), 0, _P(fake), dt, _P(fake), _P(fake), ldkv, 4, 100, 32, 128,
+                                     H, q_pos0, 8, scale, 0, _P(fake), _P(fake), None, _P(ws), 1 << 30, None)
+    assert chunk(q_pos0=97) == 1          # q_pos0 + L > N
+    assert chunk(dt=5) == 1               # unknown indexer dtype
+    assert chunk(ldkv=580) == 1           # kv rows not 16-byte aligned
+    assert chunk(H=0) == 1                # no attention heads
+    # the profiled entry point needs its events
+    assert lib.dsa_prefill_chunk_profiled(_P(fake), _P(fake), 0, _P(fake), 0, _P(fake), _P(fake), 0, 4, 100, 32,
+                                          128, 64, 96, 8, scale, 0, _P(fake), _P(fake), None, _P(ws), 1 << 30,
+                                          None, None, 0) == 1
+    # the bounded-wait self-test checks its workspace and limit before anything runs
+    assert lib.dsa_selftest_wait_timeout(None, 0, 50, None) == 3
+    assert lib.dsa_selftest_wait_timeout(_P(ws), 4096, 0, None) == 1
+    assert lib.dsa_selftest_wait_timeout(_P(ws), 4096, 5000, None) == 1
 
 
 def test_binding_refuses_cpu_tensors():
