@@ -12,8 +12,8 @@
 //     sample that LiteTopK, arXiv 2607.11976 Abstract, uses to estimate each
 //     query's score range), or
 //   * EMIT mode: compared with the query's threshold and, when it passes,
-//     appended to that query's candidate list ("write back only promising
-//     candidates", LiteTopK Abstract).
+//     appended to that query's candidate list, so that only keys able to
+//     reach the top-k are stored (LiteTopK Abstract).
 //
 // Tile shape (swap-AB): A = 128 keys x D_I (UMMA M = 128), B = a group of
 // 256 / H_I queries x H_I heads = 256 rows x D_I (UMMA N = 256), K = D_I.

@@ -1,10 +1,12 @@
 // mla.cu -- sparse absorbed-MLA attention over each query's selected keys.
 //
 // mlx-lm PR #1997 ("GLM prefill now attends only to the keys its indexer
-// picks", section "How it works"): the latent and rope caches are joined into
-// one 576-wide key per position, the top-k rows a query picked are gathered
-// once and shared by all its heads, and attention runs in the absorbed latent
-// space, so a chunk costs L * top-k instead of L * N.  For query t and head h:
+// picks", section "How it works"): each cached position holds a single key of
+// 576 values (512 latent followed by 64 rope); a query's selected rows are
+// fetched once for all of its heads; the heads attend in latent space with
+// the key projection absorbed into the query, as in decode.  The work per
+// chunk therefore grows with L * top-k rather than L * N.  For query t and
+// head h:
 //     z_j = scale * (q_lat[t,h] . kv_lat[i_j] + q_rope[t,h] . k_rope[i_j])
 //     out[t,h] = sum_j softmax(z)_j * kv_lat[i_j]          (512 wide)
 // Index -1 marks a skipped entry (llama.cpp PR #25917, discussion).

@@ -203,9 +203,9 @@ int oracle_topk_fullsort(const double *scores, int nvis, int topk, int32_t *idx_
  * Exact top-k by the blocked fold of [MLX] "How it works": score the keys in
  * blocks, fold each block into a running list of the best topk, so that each
  * selection step only looks at topk + block rows.  Must select the same set
- * as oracle_topk_fullsort (the page states the fold picks the same keys as
- * the stock indexer up to the order of equal scores; with the index
- * tie-break the sets are identical).
+ * as oracle_topk_fullsort: by the page, folding block by block can only
+ * differ from selecting over the whole row where equal scores compete for
+ * the last places, and the index tie-break removes that freedom.
  */
 int oracle_topk_blocked_fold(const double *scores, int nvis, int topk, int block, int32_t *idx_out) {
     if (nvis < 0 || topk <= 0 || block <= 0) return ORACLE_EINVAL;
