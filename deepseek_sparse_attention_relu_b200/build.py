@@ -5,6 +5,8 @@ import glob
 import os
 import subprocess
 import sys
+import tempfile
+import threading
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
@@ -36,16 +38,27 @@ def needs_build() -> bool:
     return any(os.path.getmtime(d) > t for d in deps())
 
 
+_lock = threading.Lock()
+
+
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and not needs_build():
-        return LIB
-    nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, "-o", tmp, *sources()]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
+    """Compile every csrc/*.cu into libdsa.so when a source is newer (or force).  Safe to call from
+    several threads or processes at once: each compiles to its own temporary file and renames it."""
+    with _lock:
+        if not force and not needs_build():
+            return LIB
+        nvcc = os.environ.get("NVCC", "nvcc")
+        fd, tmp = tempfile.mkstemp(prefix="libdsa.", suffix=".so.tmp", dir=PKG)
+        os.close(fd)
+        try:
+            cmd = [nvcc, *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, "-o", tmp, *sources()]
+            if verbose:
+                print(" ".join(cmd), file=sys.stderr)
+            subprocess.check_call(cmd)
+            os.replace(tmp, LIB)
+        finally:
+            if os.path.exists(tmp):
+                os.remove(tmp)
     return LIB
 
 

@@ -18,6 +18,8 @@ from __future__ import annotations
 import ctypes
 import os
 import subprocess
+import tempfile
+import threading
 from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
@@ -32,44 +34,57 @@ MLA_LAT = 512
 MLA_DIM = 576
 
 _lib = None
+_lock = threading.RLock()  # the worker threads of map_rows may all ask for the library at once
 
 
 def build(force: bool = False) -> str:
     """Compile dsa_oracle.c into liboracle.so (gcc -O2, strict IEEE: no fast-math)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(
-            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
-             _SRC, "-o", tmp, "-lm"])
-        os.replace(tmp, _LIB)
+    with _lock:
+        if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+            fd, tmp = tempfile.mkstemp(prefix="liboracle.", suffix=".so.tmp", dir=_HERE)
+            os.close(fd)
+            try:
+                subprocess.check_call(
+                    ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+                     _SRC, "-o", tmp, "-lm"])
+                os.replace(tmp, _LIB)
+            finally:
+                if os.path.exists(tmp):
+                    os.remove(tmp)
     return _LIB
 
 
 def lib() -> ctypes.CDLL:
     global _lib
-    if _lib is None:
-        build()
-        L = ctypes.CDLL(_LIB)
-        P = ctypes.c_void_p
-        i32 = ctypes.c_int
-        d = ctypes.c_double
-        L.oracle_bf16_value.restype = d
-        L.oracle_bf16_value.argtypes = [ctypes.c_uint16]
-        L.oracle_e4m3_value.restype = d
-        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
-        L.oracle_indexer_scores.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P]
-        L.oracle_indexer_scores_range.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, P]
-        L.oracle_topk_fullsort.argtypes = [P, i32, i32, P, P]
-        L.oracle_topk_blocked_fold.argtypes = [P, i32, i32, i32, P]
-        L.oracle_sparse_mla.argtypes = [P, P, P, i32, i32, i32, i32, d, i32, P, P]
-        L.oracle_dense_causal_mla.argtypes = [P, P, i32, i32, i32, i32, d, i32, P, P]
-        L.oracle_prefill_row.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, i32, d, i32,
-                                         P, P, P, P]
-        for name in ("oracle_indexer_scores", "oracle_indexer_scores_range", "oracle_topk_fullsort",
-                     "oracle_topk_blocked_fold", "oracle_sparse_mla", "oracle_dense_causal_mla", "oracle_prefill_row",
-                     "oracle_version"):
-            getattr(L, name).restype = i32
-        _lib = L
+    with _lock:
+        return _lib if _lib is not None else _load()
+
+
+def _load() -> ctypes.CDLL:
+    """Build (if stale) and load liboracle.so, declaring every entry point; called under _lock."""
+    global _lib
+    build()
+    L = ctypes.CDLL(_LIB)
+    P = ctypes.c_void_p
+    i32 = ctypes.c_int
+    d = ctypes.c_double
+    L.oracle_bf16_value.restype = d
+    L.oracle_bf16_value.argtypes = [ctypes.c_uint16]
+    L.oracle_e4m3_value.restype = d
+    L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+    L.oracle_indexer_scores.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P]
+    L.oracle_indexer_scores_range.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, P]
+    L.oracle_topk_fullsort.argtypes = [P, i32, i32, P, P]
+    L.oracle_topk_blocked_fold.argtypes = [P, i32, i32, i32, P]
+    L.oracle_sparse_mla.argtypes = [P, P, P, i32, i32, i32, i32, d, i32, P, P]
+    L.oracle_dense_causal_mla.argtypes = [P, P, i32, i32, i32, i32, d, i32, P, P]
+    L.oracle_prefill_row.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, i32, d, i32,
+                                     P, P, P, P]
+    for name in ("oracle_indexer_scores", "oracle_indexer_scores_range", "oracle_topk_fullsort",
+                 "oracle_topk_blocked_fold", "oracle_sparse_mla", "oracle_dense_causal_mla", "oracle_prefill_row",
+                 "oracle_version"):
+        getattr(L, name).restype = i32
+    _lib = L
     return _lib
 
 
