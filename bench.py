@@ -10,7 +10,9 @@ queries).  Prints one JSON line on rank 0.
 Timing: W untimed warm-up steps; then K steps, each preceded by a 512 MiB
 device write that flushes the 126 MB L2, each bracketed by CUDA events on the
 launching stream (the flush is outside the events); a barrier and a device
-synchronise on both sides of the timed region; max over ranks.  With N > 1
+synchronise on both sides of the timed region; max over ranks.  nvidia-smi
+samples clocks and throttle reasons from 0.4 s of untimed steps before the
+timed region until 0.4 s after it, so the record is taken under load.  With N > 1
 every rank runs an independent replica (the path has no cross-GPU exchange):
 value = all ranks' query tokens / max rank time (weak scaling).
 
@@ -41,6 +43,7 @@ import dsa_inputs  # noqa: E402
 METRIC = "DSA prefill query tokens/s at 128K ctx (indexer+top-k+sparse MLA); % roofline"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 512 << 20
+LOAD_WINDOW_S = 0.4  # untimed steps on each side of the timed region while the clocks are sampled
 EVENTS_PER_BLOCK = 7
 
 
@@ -81,7 +84,8 @@ def indexer_kernel_traffic(cfg) -> int | None:
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples (every 200 ms) while the timed region runs."""
+    """nvidia-smi clock / throttle-reason samples (every 200 ms) while the GPU runs the timed region and the
+    untimed load window around it."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -109,7 +113,7 @@ class ClockSampler:
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
+        time.sleep(0.05)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -131,6 +135,23 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def keep_busy(step_fn, seconds: float, sync) -> int:
+    """Run untimed steps back to back for about `seconds` of wall time (at least one), then wait for the
+    device.  Used around the timed region so that the clock sampler sees the GPU under load: the timed
+    region itself is often shorter than one sampling interval."""
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        step_fn()
+        n += 1
+        if n % 8 == 0:
+            sync()
+            if time.perf_counter() - t0 >= seconds:
+                break
+    sync()
+    return n
 
 
 def max_over_ranks(value: float, world: int, device=None) -> float:
@@ -258,7 +279,12 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     torch.cuda.synchronize()
     sampler = ClockSampler(local_rank)
     sampler.start()
-    time.sleep(0.3)
+
+    def load_step():
+        flush.zero_()
+        step(warm_ev)
+
+    keep_busy(load_step, LOAD_WINDOW_S, torch.cuda.synchronize)  # the sampler sees the GPU under load
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -268,9 +294,11 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         step(stage_ev[k])
         ends[k].record(stream)
     torch.cuda.synchronize()
+    keep_busy(load_step, LOAD_WINDOW_S, torch.cuda.synchronize)
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop()
+    clocks["window"] = f"timed steps plus {LOAD_WINDOW_S:g} s of untimed steps on each side"
     status = dsa.dsa_workspace_status(ws)
     if status != 0:
         raise RuntimeError(f"device status word {status:#x} after the timed steps")
