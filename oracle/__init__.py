@@ -26,7 +26,9 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "dsa_oracle.c")
-_LIB = os.path.join(_HERE, "liboracle.so")
+# Tests of the pins themselves point this at a prebuilt, deliberately mutated copy of the oracle.
+_OVERRIDE = os.environ.get("DSA_ORACLE_LIB")
+_LIB = _OVERRIDE or os.path.join(_HERE, "liboracle.so")
 
 IDX_BF16 = 0
 IDX_E4M3 = 1
@@ -39,6 +41,8 @@ _lock = threading.RLock()  # the worker threads of map_rows may all ask for the 
 
 def build(force: bool = False) -> str:
     """Compile dsa_oracle.c into liboracle.so (gcc -O2, strict IEEE: no fast-math)."""
+    if _OVERRIDE:
+        return _LIB
     with _lock:
         if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
             fd, tmp = tempfile.mkstemp(prefix="liboracle.", suffix=".so.tmp", dir=_HERE)
