@@ -344,7 +344,8 @@ constexpr float kMaxUnionRatio = 0.75f; // pack when the union is at most 75% of
 // adds tensor work (the rows were idle) while shared keys are gathered once.
 // Capped so the attention grid still covers the GPU at least twice.
 int pack_group(int H, int topk, int Lq, int N) {
-  if (H <= 0 || topk <= 0 || H > 32 || N > 800 * 1024) return 1;  // the pack plan's key bitmap must fit in shared memory
+  if (H <= 0 || topk <= 0) return 1;
+  if (H > 32 || N > 800 * 1024) return 1;  // the pack plan's key bitmap must fit in shared memory
   int G = std::min(64 / H, 8);  // the attention kernel tracks up to 8 queries per CTA
   G = std::min(G, kPackMaxEntries / topk);
   G = std::min(G, std::max(1, Lq / (2 * std::max(1, sm_count()))));
