@@ -28,9 +28,15 @@ EXPORTED = ("dsa_version", "dsa_status_string", "dsa_last_error_string", "dsa_in
             "dsa_sparse_mla_workspace", "dsa_sparse_mla_prefill", "dsa_prefill_chunk_workspace",
             "dsa_prefill_chunk", "dsa_prefill_chunk_profiled", "dsa_workspace_status",
             "dsa_indexer_topk_noalloc", "dsa_indexer_topk_ranges", "dsa_prefill_chunk_ranges",
-            "dsa_selftest_wait_timeout")
+            "dsa_selftest_wait_timeout", "dsa_indexer_topk_noalloc_status", "dsa_workspace_selection_stats")
 
 _lib = None
+
+
+class SelectionStats(ctypes.Structure):
+    """dsa_selection_stats_t (include/dsa.h)."""
+    _fields_ = [("candidates", ctypes.c_ulonglong), ("queries", ctypes.c_uint), ("fallback_queries", ctypes.c_uint),
+                ("max_candidates", ctypes.c_uint), ("reserved", ctypes.c_uint)]
 
 
 class DSAError(RuntimeError):
@@ -84,6 +90,10 @@ def lib() -> ctypes.CDLL:
         L.dsa_selftest_wait_timeout.argtypes = [P, Z, ctypes.c_uint, P]
         L.dsa_workspace_status.restype = I
         L.dsa_workspace_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint)]
+        L.dsa_indexer_topk_noalloc_status.restype = I
+        L.dsa_workspace_selection_stats.restype = I
+        L.dsa_workspace_selection_stats.argtypes = [P, P, ctypes.POINTER(SelectionStats)]
+        L.dsa_indexer_topk_noalloc_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
         _lib = L
     return _lib
 
@@ -199,11 +209,12 @@ def dsa_indexer_topk_ranges(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.T
 
 def dsa_indexer_topk_noalloc(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, q_pos0: int, topk: int,
                              topk_idx: torch.Tensor, topk_score: torch.Tensor | None = None, stream=None) -> None:
-    """dsa_indexer_topk without a workspace, for callers that cannot allocate device memory (inside CUDA graph
-    capture, under a runtime that plans all memory up front, or on a fully reserved device).  The scratch is a
-    fixed 16 MiB array inside libdsa.so shared by every call on the device: calls that overlap on the GPU race,
-    and problems too large for it raise DSAError(DSA_ERR_WORKSPACE).  The first call on a device looks up the
-    array's address, so make it before any stream capture."""
+    """dsa_indexer_topk without a workspace, for callers that cannot allocate device memory (a runtime that
+    plans all memory up front and hands kernels only their inputs and outputs, or a device fully reserved by
+    others).  The scratch is a fixed 16 MiB array inside libdsa.so shared by every call on the device: calls
+    that overlap on the GPU race, and problems too large for it raise DSAError(DSA_ERR_WORKSPACE).  The first
+    call on a device looks up the array's address, so make it before any stream capture.  Device-side
+    conditions are read with dsa_indexer_topk_noalloc_status()."""
     L, H_I, D_I = q_idx.shape
     N = k_idx.shape[0]
     dt = _dtype_code(q_idx)
@@ -307,6 +318,26 @@ def dsa_selftest_wait_timeout(workspace: torch.Tensor, limit_ms: int = 50, strea
     """Run the bounded-wait self-test into `workspace` (see include/dsa.h); read it with dsa_workspace_status."""
     _check(lib().dsa_selftest_wait_timeout(_dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                                            int(limit_ms), _stream(stream)), "dsa_selftest_wait_timeout")
+
+
+def dsa_indexer_topk_noalloc_status(stream=None) -> int:
+    """Synchronise the stream and return the status word of dsa_indexer_topk_noalloc's fixed scratch on the
+    current device (0 = clean; it describes the most recent call)."""
+    flags = ctypes.c_uint(0)
+    st = lib().dsa_indexer_topk_noalloc_status(_stream(stream), ctypes.byref(flags))
+    if st not in (DSA_OK, 5):
+        raise DSAError(st, "dsa_indexer_topk_noalloc_status")
+    return flags.value
+
+
+def dsa_workspace_selection_stats(workspace: torch.Tensor, stream=None) -> dict:
+    """Synchronise the stream and return the selection totals of the most recent call on `workspace`:
+    candidates (all queries), queries, fallback_queries, max_candidates."""
+    s = SelectionStats()
+    _check(lib().dsa_workspace_selection_stats(_dev(workspace, "workspace"), _stream(stream), ctypes.byref(s)),
+           "dsa_workspace_selection_stats")
+    return {"candidates": s.candidates, "queries": s.queries, "fallback_queries": s.fallback_queries,
+            "max_candidates": s.max_candidates}
 
 
 def dsa_workspace_status(workspace: torch.Tensor, stream=None) -> int:

@@ -21,7 +21,9 @@ constexpr int kSamples = 4096;            // strided key sample per query block
 constexpr int kFallbackSlots = 16;        // CTAs (and score rows) of the exact fallback
 constexpr int kMinCap = 8192;             // default candidate capacity per query
 constexpr int kMaxTopk = 4096;
-constexpr size_t kHeaderBytes = 256;      // status word, fallback counters
+constexpr size_t kHeaderBytes = 256;      // status word, fallback counters, selection totals
+constexpr size_t kStatsOffset = 32;       // selection totals in the header
+static_assert(sizeof(dsa::SelectionStats) == sizeof(dsa_selection_stats_t), "stats layout");
 
 // The CUDA error behind the calling thread's last DSA_ERR_CUDA (cudaSuccess if none).
 thread_local cudaError_t t_last_cuda_error = cudaSuccess;
@@ -80,6 +82,18 @@ int sm_count() {
 
 int default_cap(int topk) { return std::max(kMinCap, 4 * topk); }
 
+// Queries per block: the caller's query_block (<= 0: 1,024), rounded up to a
+// whole number of indexer query groups (256 / H_I queries share one tensor-core
+// tile), at most L.  Every query then sits in the same group tile, at the same
+// column, whatever the blocking, so its scores -- and its selection -- do not
+// depend on the blocking.
+int query_block_size(int L, int query_block, int H_I) {
+  const int qg = (H_I > 0 && 256 % H_I == 0) ? 256 / H_I : 1;
+  long long qb = query_block > 0 ? query_block : kDefaultQueryBlock;
+  qb = (qb + qg - 1) / qg * qg;
+  return static_cast<int>(std::min<long long>(L, qb));
+}
+
 // Fixed part of the indexer workspace (everything but the candidate lists).
 size_t idx_fixed_bytes(int QB, int N) {
   return kHeaderBytes + 5 * align256(static_cast<size_t>(QB) * 4) + 2 * align256((QB + 2) * sizeof(int)) +
@@ -89,6 +103,7 @@ size_t idx_fixed_bytes(int QB, int N) {
 struct IdxWorkspace {
   unsigned *status;
   int *fb_counters;
+  SelectionStats *stats;
   unsigned *tau;
   int *cand_count;
   int *fb_list;
@@ -106,6 +121,7 @@ bool carve_idx_ws(void *ws, size_t bytes, int QB, int N, IdxWorkspace *o) {
   uint8_t *p = static_cast<uint8_t *>(ws);
   o->status = reinterpret_cast<unsigned *>(p);
   o->fb_counters = reinterpret_cast<int *>(p + 16);
+  o->stats = reinterpret_cast<SelectionStats *>(p + kStatsOffset);
   p += kHeaderBytes;
   o->tau = reinterpret_cast<unsigned *>(p);
   p += align256(static_cast<size_t>(QB) * 4);
@@ -234,29 +250,24 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
     pa.dense_ld = n_samples;
     pa.n_keys = n_samples;
     pa.total_tiles = G * ((n_samples + 127) / 128);
-    if (!cuda_ok(launch_indexer(tq, ts, pa, p.D_I, p.H_I, p.fp8, true, std::min(sms, pa.total_tiles), stream)))
+    if (!cuda_ok(launch_indexer(tq, ts, pa, p.D_I, p.H_I, p.fp8, kIdxPilot, std::min(sms, pa.total_tiles), stream)))
       return DSA_ERR_CUDA;
   }
 
   SelectArgs sa{};
-  sa.q_idx = p.q_idx;
-  sa.k_idx = p.k_idx;
-  sa.ldk = p.key_ld();
-  sa.w = p.w;
   sa.dense = pilot ? ws.dense : nullptr;
   sa.tau = ws.tau;
   sa.cand = ws.cand;
   sa.cand_count = ws.cand_count;
   sa.fb_list = ws.fb_list;
   sa.fb_counters = ws.fb_counters;
-  sa.fb_scratch = ws.fb_scratch;
   sa.status = ws.status;
+  sa.stats = ws.stats;
   sa.topk_idx = p.topk_idx;
   sa.topk_score = p.topk_score;
   sa.dense_ld = n_samples;
   sa.n_samples = n_samples;
   sa.cap = ws.cap;
-  sa.fb_slots = kFallbackSlots;
   sa.t0 = t0;
   sa.Lb = Lb;
   sa.q_pos0 = q_pos0;
@@ -264,10 +275,7 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
   sa.key_hi = ranges ? ws.rhi : nullptr;
   sa.sample_stride = static_cast<int>(stride);
   sa.N = p.N;
-  sa.H_I = p.H_I;
-  sa.D_I = p.D_I;
   sa.topk = p.topk;
-  sa.fp8 = p.fp8 ? 1 : 0;
   if (!mark(ev, 1, stream)) return DSA_ERR_CUDA;
   if (!cuda_ok(launch_threshold(sa, stream))) return DSA_ERR_CUDA;
   if (!mark(ev, 2, stream)) return DSA_ERR_CUDA;
@@ -287,13 +295,26 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
   }
   if (total > (1ll << 30)) return DSA_ERR_UNSUPPORTED;
   ea.total_tiles = static_cast<int>(total);
-  if (!cuda_ok(launch_indexer(tq, tk, ea, p.D_I, p.H_I, p.fp8, false,
+  if (!cuda_ok(launch_indexer(tq, tk, ea, p.D_I, p.H_I, p.fp8, kIdxEmit,
                               static_cast<int>(std::min<long long>(sms, total)), stream)))
     return DSA_ERR_CUDA;
   if (!mark(ev, 3, stream)) return DSA_ERR_CUDA;
   if (!cuda_ok(launch_select(sa, stream))) return DSA_ERR_CUDA;
   if (!mark(ev, 4, stream)) return DSA_ERR_CUDA;
-  if (!cuda_ok(launch_fallback(sa, stream))) return DSA_ERR_CUDA;
+  // Exact fallback for the queries the selection handed over: the indexer
+  // kernel rescores each of them over all its visible keys with the main
+  // pass's arithmetic (same group tile, same key tiles) into a dense row and
+  // selects from it.  With no such query its CTAs exit at once.
+  IndexerArgs fa = ea;
+  fa.dense = ws.fb_scratch;
+  fa.dense_ld = p.N;
+  fa.fb_list = ws.fb_list;
+  fa.fb_counters = ws.fb_counters;
+  fa.topk_idx = p.topk_idx + static_cast<long long>(t0) * p.topk;
+  fa.topk_score = p.topk_score ? p.topk_score + static_cast<long long>(t0) * p.topk : nullptr;
+  fa.topk = p.topk;
+  if (!cuda_ok(launch_indexer(tq, tk, fa, p.D_I, p.H_I, p.fp8, kIdxFallback, kFallbackSlots, stream)))
+    return DSA_ERR_CUDA;
   if (!mark(ev, 5, stream)) return DSA_ERR_CUDA;
   return DSA_OK;
 }
@@ -342,14 +363,19 @@ constexpr float kMaxUnionRatio = 0.75f; // pack when the union is at most 75% of
 // Queries packed per CTA: with H <= 32 heads a 64-row tile has room for
 // 64 / H queries, and packing them over the union of their selections never
 // adds tensor work (the rows were idle) while shared keys are gathered once.
-// Capped so the attention grid still covers the GPU at least twice.
-int pack_group(int H, int topk, int Lq, int N) {
+// Capped so the attention grid still covers the GPU at least twice.  Decided
+// from the whole chunk's L (never a query block's) and rounded down to a power
+// of two, so that packs, which start at a block's first query, are the same
+// for every blocking (blocks are whole multiples of 8 queries).
+int pack_group(int H, int topk, int L, int N) {
   if (H <= 0 || topk <= 0) return 1;
   if (H > 32 || N > 800 * 1024) return 1;  // the pack plan's key bitmap must fit in shared memory
   int G = std::min(64 / H, 8);  // the attention kernel tracks up to 8 queries per CTA
   G = std::min(G, kPackMaxEntries / topk);
-  G = std::min(G, std::max(1, Lq / (2 * std::max(1, sm_count()))));
-  return std::max(G, 1);
+  G = std::min(G, std::max(1, L / (2 * std::max(1, sm_count()))));
+  G = std::max(G, 1);
+  while (G & (G - 1)) G &= G - 1;  // largest power of two <= G
+  return G;
 }
 
 // Union buffers for up to Lq queries packed G at a time (any G).
@@ -421,7 +447,7 @@ dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, unsigned 
     if (!cuda_ok(launch_sparse_mla(tq, a, false, stream))) return DSA_ERR_CUDA;
     return cuda_ok(launch_mla_combine(a, stream)) ? DSA_OK : DSA_ERR_CUDA;
   }
-  const int G = pack_group(p.H, p.topk, Lq, p.N);
+  const int G = pack_group(p.H, p.topk, p.L, p.N);
   if (G >= 2 && uw.base != nullptr && uw.bytes >= union_bytes(Lq, p.topk)) {
     const int npacks = (Lq + G - 1) / G;
     const int umax = (G * p.topk + 63) / 64 * 64;  // whole 64-key tiles
@@ -490,7 +516,7 @@ const char *dsa_status_string(dsa_status_t s) {
 size_t dsa_indexer_topk_workspace(int L, int N, int H_I, int D_I, int topk, dsa_dtype_t dtype) {
   if (L <= 0 || N <= 0 || H_I <= 0 || D_I <= 0 || topk <= 0) return 0;
   (void)dtype;
-  const int QB = std::min(L, kDefaultQueryBlock);
+  const int QB = query_block_size(L, 0, H_I);
   return idx_fixed_bytes(QB, N) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
 }
 
@@ -509,7 +535,7 @@ dsa_status_t indexer_topk_impl(const void *q_idx, const void *k_idx, int64_t ldk
   p.ldk = ldk;
   dsa_status_t st = check_indexer_args(p);
   if (st != DSA_OK) return st;
-  const int QB = std::min(L, kDefaultQueryBlock);
+  const int QB = query_block_size(L, 0, H_I);
   IdxWorkspace ws;
   if (!carve_idx_ws(workspace, workspace_bytes, QB, N, &ws)) return DSA_ERR_WORKSPACE;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
@@ -571,7 +597,7 @@ size_t dsa_prefill_chunk_workspace(int L, int N, int H_I, int D_I, int H, int to
                                    dsa_dtype_t dtype, int want_topk_out) {
   if (L <= 0 || N <= 0 || H_I <= 0 || D_I <= 0 || H <= 0 || topk <= 0) return 0;
   (void)dtype;
-  const int QB = std::min(L, query_block > 0 ? query_block : kDefaultQueryBlock);
+  const int QB = query_block_size(L, query_block, H_I);
   size_t bytes = idx_fixed_bytes(QB, N) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
   if (!want_topk_out) bytes += align256(static_cast<size_t>(QB) * topk * 4);
   const size_t extra = attention_scratch_bytes(L, QB, H, topk);
@@ -591,7 +617,7 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, int64_t ld
   if (dtype != DSA_BF16 && dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID_ARG;
   // Sizes first: the scratch planning below divides by them.
   if (L <= 0 || N <= 0 || H_I <= 0 || D_I <= 0 || H <= 0 || topk <= 0) return DSA_ERR_INVALID_ARG;
-  const int QB = std::min(L, query_block > 0 ? query_block : kDefaultQueryBlock);
+  const int QB = query_block_size(L, query_block, H_I);
   // Selected keys: the caller's buffer, or a block-sized region at the end of the workspace.
   size_t idx_bytes = workspace_bytes;
   int32_t *block_idx = nullptr;
@@ -697,6 +723,17 @@ dsa_status_t dsa_selftest_wait_timeout(void *workspace, size_t workspace_bytes, 
              : DSA_ERR_CUDA;
 }
 
+dsa_status_t dsa_workspace_selection_stats(const void *workspace, dsa_stream_t stream_,
+                                           dsa_selection_stats_t *stats) {
+  if (workspace == nullptr || stats == nullptr) return DSA_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!cuda_ok(cudaStreamSynchronize(stream))) return DSA_ERR_CUDA;
+  if (!cuda_ok(cudaMemcpy(stats, static_cast<const uint8_t *>(workspace) + kStatsOffset, sizeof(*stats),
+                          cudaMemcpyDeviceToHost)))
+    return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
 dsa_status_t dsa_workspace_status(const void *workspace, dsa_stream_t stream_, unsigned *flags) {
   if (workspace == nullptr || flags == nullptr) return DSA_ERR_INVALID_ARG;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
@@ -714,7 +751,8 @@ dsa_status_t dsa_workspace_status(const void *workspace, dsa_stream_t stream_, u
 // device memory (see include/dsa.h).  Its scratch is this file-scope device
 // array, held by every GPU that loads the library until the process exits.
 // Host code cannot use the array's name as a device address: the address is
-// looked up once per device with cudaGetSymbolAddress and passed on.
+// looked up with cudaGetSymbolAddress, with the device current, the first time
+// a device (more exactly, a CUDA context on it) is used, and passed on.
 // ---------------------------------------------------------------------------
 #include <mutex>
 
@@ -726,22 +764,58 @@ constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_noalloc_mutex;
-void *g_noalloc_addr[kNoAllocMaxDevices] = {};
+// Identity of the calling thread's current CUDA context (0 if there is none
+// or the driver cannot tell).  A device reset or a re-created primary context
+// gets a new identity, and the library's module -- with the array -- may then
+// sit elsewhere, so the cached address is keyed on it.
+unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext *);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long *);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
-// Device address of the scratch array on the current device; the first call
-// per device does the lookup.
+struct NoAllocEntry {
+  void *addr = nullptr;
+  unsigned long long ctx_id = 0;
+};
+std::mutex g_noalloc_mutex;
+NoAllocEntry g_noalloc[kNoAllocMaxDevices];
+
+// Device address of the scratch array in the current device's context.  The
+// lookup runs on the first call in a context (and on every call if the
+// context's identity cannot be read).
 dsa_status_t noalloc_scratch(void **out) {
   int dev = 0;
   if (!cuda_ok(cudaGetDevice(&dev))) return DSA_ERR_CUDA;
   if (dev < 0 || dev >= kNoAllocMaxDevices) return DSA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[dev] == nullptr) {
+  NoAllocEntry &e = g_noalloc[dev];
+  const unsigned long long id = current_context_id();
+  if (e.addr == nullptr || id == 0 || id != e.ctx_id) {
     void *p = nullptr;
     if (!cuda_ok(cudaGetSymbolAddress(&p, g_noalloc_scratch))) return DSA_ERR_CUDA;
-    g_noalloc_addr[dev] = p;
+    e.addr = p;
+    e.ctx_id = current_context_id();  // the lookup may have created the context
   }
-  *out = g_noalloc_addr[dev];
+  *out = e.addr;
   return DSA_OK;
 }
 
@@ -756,7 +830,7 @@ extern "C" dsa_status_t dsa_indexer_topk_noalloc(const void *q_idx, const void *
   p.ldk = ldk;
   dsa_status_t st = check_indexer_args(p);
   if (st != DSA_OK) return st;
-  const int QB = std::min(L, kNoAllocQueryBlock);
+  const int QB = query_block_size(L, kNoAllocQueryBlock, H_I);
   // Too large for the fixed scratch: refuse before touching the device.
   if (idx_fixed_bytes(QB, N) + static_cast<size_t>(QB) * default_cap(topk) * 8 > kNoAllocScratchBytes)
     return DSA_ERR_WORKSPACE;
@@ -776,4 +850,17 @@ extern "C" dsa_status_t dsa_indexer_topk_noalloc(const void *q_idx, const void *
     if (st != DSA_OK) return st;
   }
   return DSA_OK;
+}
+
+extern "C" dsa_status_t dsa_indexer_topk_noalloc_status(dsa_stream_t stream_, unsigned *flags) {
+  if (flags == nullptr) return DSA_ERR_INVALID_ARG;
+  void *scratch = nullptr;
+  const dsa_status_t st = noalloc_scratch(&scratch);
+  if (st != DSA_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  unsigned v = 0;
+  if (!cuda_ok(cudaStreamSynchronize(stream))) return DSA_ERR_CUDA;
+  if (!cuda_ok(cudaMemcpy(&v, scratch, sizeof(v), cudaMemcpyDeviceToHost))) return DSA_ERR_CUDA;
+  *flags = v;
+  return v == 0 ? DSA_OK : DSA_ERR_INTERNAL;
 }

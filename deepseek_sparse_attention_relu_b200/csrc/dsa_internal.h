@@ -47,6 +47,15 @@ struct IndexerArgs {
   int q_row0;                     // first row of the block in the [L*H_I, D_I] query tensor map
   int total_tiles;                // sum over query groups of their 128-key tiles
   int pilot;                      // 1 = PILOT mode
+  // FALLBACK mode: the CTAs take the queries of fb_list[0 .. fb_counters[0])
+  // one at a time (fb_counters[1] hands them out), score every visible key of
+  // the query into their own dense row of `dense` (dense_ld = N floats per
+  // CTA) and select its exact top-k into topk_idx / topk_score.
+  const int *fb_list;             // [Lb] queries of the block, as positions tl
+  int *fb_counters;               // [0] = count, [1] = next
+  int32_t *topk_idx;              // [Lb, topk] rows of the block's queries
+  float *topk_score;              // [Lb, topk] or nullptr
+  int topk;
   // Per-query key ranges (general causality; nullptr = causal, query tl sees
   // keys <= q_pos0 + tl): query tl of the block sees keys key_lo[tl] <=
   // s < key_hi[tl].  Then group g covers the 128-key tiles grp_tile0[g] ..
@@ -69,37 +78,47 @@ struct RangePlanArgs {
 cudaError_t launch_range_plan(const RangePlanArgs &a, cudaStream_t stream);
 cudaError_t launch_wait_timeout_probe(unsigned *status, unsigned long long limit_ns, cudaStream_t stream);
 
+// Modes of the indexer kernel: every visible score compared with the query's
+// threshold (EMIT), dense scores of a key sample (PILOT), or the exact
+// fallback for the queries the selection could not resolve (FALLBACK).
+enum IndexerMode : int { kIdxEmit = 0, kIdxPilot = 1, kIdxFallback = 2 };
+
 cudaError_t launch_indexer(const CUtensorMap &tq, const CUtensorMap &tk, const IndexerArgs &a, int D_I, int H_I,
-                           bool fp8, bool pilot, int grid, cudaStream_t stream);
+                           bool fp8, IndexerMode mode, int grid, cudaStream_t stream);
 bool indexer_supported(int D_I, int H_I, bool fp8);
 int indexer_queries_per_group(int H_I);
 
-// Threshold / selection / fallback stage.
+// Selection totals of one call, accumulated by the selection kernel over all
+// query blocks (in the workspace header; layout of dsa_selection_stats_t).
+struct SelectionStats {
+  unsigned long long candidates;  // candidate keys found over all queries (before the capacity cut)
+  unsigned queries;               // queries selected
+  unsigned fallback_queries;      // queries resolved by the exact fallback
+  unsigned max_candidates;        // largest candidate count of one query
+  unsigned pad;
+};
+
+// Threshold / selection stage.
 struct SelectArgs {
-  const void *q_idx;              // [L, H_I, D_I] whole chunk (fallback rescoring)
-  const void *k_idx;              // [N, D_I]
-  const float *w;                 // [L, H_I] whole chunk
   const float *dense;             // [Lb, dense_ld] pilot sample scores, or nullptr
   unsigned *tau;                  // [Lb] threshold score keys
   const unsigned long long *cand; // [Lb, cap]
   int *cand_count;                // [Lb]
   int *fb_list;                   // [Lb] queries that need the exact fallback
   int *fb_counters;               // [0] = count, [1] = next
-  float *fb_scratch;              // [fb_slots, N] fallback score rows
   unsigned *status;
+  SelectionStats *stats;          // totals over the call (workspace header)
   int32_t *topk_idx;              // [L, topk] whole chunk
   float *topk_score;              // [L, topk] or nullptr
-  int dense_ld, n_samples, cap, fb_slots;
-  long long ldk;                  // k_idx row stride in elements
+  int dense_ld, n_samples, cap;
   const int *key_lo, *key_hi;     // [Lb] clamped per-query ranges, or nullptr (causal)
   int sample_stride;              // with ranges: pilot sample i is key i * sample_stride
   int t0, Lb, q_pos0;             // block: first query (chunk row), size, position of first query
-  int N, H_I, D_I, topk, fp8;
+  int N, topk;
 };
 
 cudaError_t launch_threshold(const SelectArgs &a, cudaStream_t stream);
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream);
-cudaError_t launch_fallback(const SelectArgs &a, cudaStream_t stream);
 
 // Sparse absorbed-MLA attention.
 struct MlaArgs {
@@ -146,6 +165,9 @@ struct PackArgs {
 cudaError_t launch_pack_plan(const PackArgs &a, cudaStream_t stream);
 
 cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, bool packed, cudaStream_t stream);
+// The unpacked attention on CTA pairs (the 576-wide contraction split over a
+// cluster of two CTAs); no work list.
+cudaError_t launch_sparse_mla_pair(const CUtensorMap &tq, const MlaArgs &a, cudaStream_t stream);
 cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t stream);
 
 }  // namespace dsa

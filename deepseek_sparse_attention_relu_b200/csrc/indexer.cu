@@ -32,6 +32,7 @@
 
 #include "dsa_internal.h"
 #include "ptx.cuh"
+#include "select_common.cuh"
 
 namespace dsa {
 
@@ -176,12 +177,32 @@ __device__ __forceinline__ void idx_cursor_next(TileCursor &c, const IndexerArgs
   }
 }
 
-template <int DI, int HI, bool FP8, bool PILOT, bool RANGES>
+// Tiles of one fallback job: every 128-key tile holding a visible key of query
+// tl (its clamped range, or its causal prefix), within the query's group.  The
+// tiles sit at the same 128-key boundaries, and the query at the same column
+// of the same group tile, as in the main pass, so its scores come out
+// bit-identical to the main pass's.
+template <bool RANGES>
+__device__ __forceinline__ TileCursor idx_cursor_job(const IndexerArgs &a, int tl, int QG, int &lo, int &hi) {
+  lo = RANGES ? a.key_lo[tl] : 0;
+  hi = RANGES ? a.key_hi[tl] : min(a.n_keys, a.q_pos0 + tl + 1);
+  TileCursor c;
+  c.g = tl / QG;
+  c.tile = 0;
+  c.tile0 = lo / 128;
+  c.ntiles_g = hi > lo ? (hi - 1) / 128 - lo / 128 + 1 : 0;
+  c.left = c.ntiles_g;
+  return c;
+}
+
+template <int DI, int HI, bool FP8, int MODE, bool RANGES>
 __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    IndexerArgs a) {
   pdl_wait_and_release();
   using C = IdxCfg<DI, HI, FP8>;
+  constexpr bool PILOT = MODE == kIdxPilot;
+  constexpr bool FB = MODE == kIdxFallback;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *q_s = smem + C::OFF_Q;
@@ -198,6 +219,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
   uint64_t *drain = q_full + 6;             // MMA drain on abort
   unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + C::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
+  volatile int *job_s = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 12);  // FALLBACK: current query
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -230,307 +252,358 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
   tc_fence_after();
   const unsigned tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      TileCursor c = idx_cursor_begin<RANGES>(a, C::QG);
-      int stage = 0;
-      unsigned phase = 0, qphase = 0;
-      int prev_g = -1, issued = 0, q_issued = 0;
-      bool ok = true;
-      while (c.left > 0) {
-        if (c.g != prev_g) {
-          if (prev_g >= 0) {
-            if (!mbar_wait(q_empty, qphase, abort_flag)) { ok = false; break; }
-            qphase ^= 1u;
-          }
-          mbar_arrive_expect_tx(q_full, C::Q_TILE);
-          for (int at = 0; at < C::ATOMS; ++at)
-            tma_load_2d(q_s + at * C::BN * 128, &tmap_q, q_full, at * C::ATOM_ELEMS, a.q_row0 + c.g * C::BN);
-          ++q_issued;
-          prev_g = c.g;
+  // ---- role state; it carries over from one fallback job to the next (the
+  // other modes make a single pass over the CTA's share of the tiles).
+  // TMA producer (warp 0, lane 0)
+  int p_stage = 0, p_issued = 0, p_q_issued = 0;
+  unsigned p_phase = 0, p_qphase = 0;
+  bool p_ok = true;
+  // MMA issuer (warp 1)
+  int m_stage = 0, m_acc = 0;
+  unsigned m_phase = 0, m_acc_phase = 0, m_qphase = 0;
+  bool m_ok = true;
+  // epilogue (warps 2..17)
+  const int ew = warp - 2;          // 0..15
+  const int quarter = warp & 3;     // TMEM lane quarter this warp may access
+  const int slot = ew >> 2;         // which 64 accumulator columns
+  constexpr int QH = C::QH;         // queries per warp
+  constexpr int SB = C::SB;
+  int e_acc = 0, e_prev_g = -1;
+  unsigned e_acc_phase = 0;
+  bool e_ok = true;
+  const unsigned lane_mask_lt = (1u << lane) - 1u;
+  float *w_w = w_s + ew * C::COLS;   // this warp's head weights: [QH queries][HI]
+  float *tau_w = tau_s + ew * C::COLS;
+  int *lo_w = reinterpret_cast<int *>(tau_w + QH);      // per-query key ranges (ranges mode)
+  int *hi_w = reinterpret_cast<int *>(tau_w + 2 * QH);
+  static_assert(3 * C::QH <= C::COLS, "thresholds and ranges share the per-warp slot");
+  unsigned long long *stg = reinterpret_cast<unsigned long long *>(smem + C::OFF_STG) + ew * QH * SB;
+  int cnt[QH];                   // staged candidates per query (warp-uniform)
+  // Indexer heads in whole 8-column blocks: 16-lane accumulator loads with the
+  // warp's head weights held in registers for the whole query group.
+  constexpr bool QUAD = (HI % 8) == 0;
+  const int c4 = lane & 3, r4 = lane >> 2;
+  float2 wreg[QH][HI / 8 > 0 ? HI / 8 : 1];
+#pragma unroll
+  for (int qq = 0; qq < QH; ++qq) cnt[qq] = 0;
+
+  // Move a query's staged candidates to its global list: one atomic per batch.
+  auto flush = [&](int qq, int gq) {
+    const int n = cnt[qq];
+    if (n == 0) return;
+    const int tl = gq * C::QG + slot * QH + qq;
+    __syncwarp();
+    int base = 0;
+    if (lane == 0) base = atomicAdd(&a.cand_count[tl], n);
+    base = __shfl_sync(0xffffffffu, base, 0);
+    for (int i = lane; i < n; i += 32) {
+      const int pos = base + i;
+      if (pos < a.cap) a.cand[static_cast<long long>(tl) * a.cap + pos] = stg[qq * SB + i];
+    }
+    __syncwarp();
+    cnt[qq] = 0;
+  };
+
+  for (int round = 0;; ++round) {
+    // ---- the tiles of this round: the CTA's share of the block (one round),
+    // or one fallback query at a time.
+    TileCursor c;
+    int job_tl = -1, job_lo = 0, job_hi = 0;
+    if constexpr (FB) {
+      if (threadIdx.x == 0) {
+        int j = -1;
+        if (!*abort_flag) {
+          const int n = atomicAdd(&a.fb_counters[1], 1);
+          if (n < *reinterpret_cast<volatile int *>(&a.fb_counters[0])) j = a.fb_list[n];
         }
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full[stage], C::K_TILE);
-        for (int at = 0; at < C::ATOMS; ++at)
-          tma_load_2d(k_s + stage * C::K_TILE + at * C::BM * 128, &tmap_k, &full[stage], at * C::ATOM_ELEMS,
-                      c.key0());
-        ++issued;
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
-        idx_cursor_next<RANGES>(c, a, C::QG);
+        *job_s = j;
       }
-      if (!ok) {
+      __syncthreads();
+      job_tl = *job_s;
+      if (job_tl < 0) break;
+      c = idx_cursor_job<RANGES>(a, job_tl, C::QG, job_lo, job_hi);
+      e_prev_g = -1;  // every job loads its group's weights afresh
+    } else {
+      if (round > 0) break;
+      c = idx_cursor_begin<RANGES>(a, C::QG);
+    }
+
+    if (warp == 0) {
+      // ---------------------------------------------------------- TMA producer
+      if (lane == 0 && p_ok) {
+        int prev_g = -1;
+        while (c.left > 0) {
+          if (c.g != prev_g) {
+            if (p_q_issued > 0) {
+              if (!mbar_wait(q_empty, p_qphase, abort_flag)) { p_ok = false; break; }
+              p_qphase ^= 1u;
+            }
+            mbar_arrive_expect_tx(q_full, C::Q_TILE);
+            for (int at = 0; at < C::ATOMS; ++at)
+              tma_load_2d(q_s + at * C::BN * 128, &tmap_q, q_full, at * C::ATOM_ELEMS, a.q_row0 + c.g * C::BN);
+            ++p_q_issued;
+            prev_g = c.g;
+          }
+          if (!mbar_wait(&empty[p_stage], p_phase ^ 1u, abort_flag)) { p_ok = false; break; }
+          mbar_arrive_expect_tx(&full[p_stage], C::K_TILE);
+          for (int at = 0; at < C::ATOMS; ++at)
+            tma_load_2d(k_s + p_stage * C::K_TILE + at * C::BM * 128, &tmap_k, &full[p_stage], at * C::ATOM_ELEMS,
+                        c.key0());
+          ++p_issued;
+          if (++p_stage == C::STAGES) { p_stage = 0; p_phase ^= 1u; }
+          idx_cursor_next<RANGES>(c, a, C::QG);
+        }
+        if (!p_ok) {
+          atomicOr(a.status, DEV_TIMEOUT);
+          *abort_flag = 1;
+        }
+      }
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr unsigned idesc = make_idesc(C::BM, C::BN, FP8 ? 0u : 1u, 0u, 0u);
+      int prev_g = -1;
+      while (m_ok && c.left > 0) {
+        const int g = c.g;
+        if (g != prev_g) {
+          if (!mbar_wait(q_full, m_qphase, abort_flag)) { m_ok = false; break; }
+          m_qphase ^= 1u;
+          prev_g = g;
+        }
+        if (!mbar_wait(&full[m_stage], m_phase, abort_flag)) { m_ok = false; break; }
+        if (!mbar_wait(&acc_empty[m_acc], m_acc_phase ^ 1u, abort_flag)) { m_ok = false; break; }
+        tc_fence_after();
+        TileCursor nx = c;
+        idx_cursor_next<RANGES>(nx, a, C::QG);
+        const bool last_of_group = (nx.left == 0) || (nx.g != g);
+        if (lane == 0) {
+          const unsigned d_tmem = tmem_base + m_acc * 256;
+          const uint64_t a0 = smem_desc_sw128(smem_u32(k_s + m_stage * C::K_TILE), 16, 1024);
+          const uint64_t b0 = smem_desc_sw128(smem_u32(q_s), 16, 1024);
+#pragma unroll
+          for (int at = 0; at < C::ATOMS; ++at) {
+#pragma unroll
+            for (int ks = 0; ks < C::KSTEPS_PER_ATOM; ++ks) {
+              // offsets go into the start-address field (address >> 4), which cannot carry
+              const uint64_t ad = a0 + static_cast<uint64_t>((at * C::BM * 128 + ks * 32) >> 4);
+              const uint64_t bd = b0 + static_cast<uint64_t>((at * C::BN * 128 + ks * 32) >> 4);
+              const unsigned accum = (at | ks) ? 1u : 0u;
+              if (FP8)
+                mma_fp8_ss(d_tmem, ad, bd, idesc, accum);
+              else
+                mma_bf16_ss(d_tmem, ad, bd, idesc, accum);
+            }
+          }
+          tc_commit(&empty[m_stage]);
+          tc_commit(&acc_full[m_acc]);
+          if (last_of_group) tc_commit(q_empty);
+        }
+        __syncwarp();
+        if (++m_stage == C::STAGES) { m_stage = 0; m_phase ^= 1u; }
+        if (++m_acc == 2) { m_acc = 0; m_acc_phase ^= 1u; }
+        c = nx;
+      }
+      if (!m_ok && lane == 0) {
         atomicOr(a.status, DEV_TIMEOUT);
         *abort_flag = 1;
       }
-      // Never leave with copies in flight.  Only the last STAGES issued tiles can
-      // still be landing, and each of them is the final use of its stage, so the
-      // phase parity below is unambiguous (an older phase of a reused stage would
-      // alias the current, never-completing one).
-      bool drained = true;
-      for (int i = (issued > C::STAGES ? issued - C::STAGES : 0); i < issued; ++i)
-        drained &= mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1u, nullptr);
-      if (q_issued > 0) drained &= mbar_wait(q_full, static_cast<unsigned>(q_issued - 1) & 1u, nullptr);
-      if (!drained) atomicOr(a.status, DEV_TIMEOUT);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    TileCursor c = idx_cursor_begin<RANGES>(a, C::QG);
-    constexpr unsigned idesc = make_idesc(C::BM, C::BN, FP8 ? 0u : 1u, 0u, 0u);
-    int stage = 0, acc = 0, prev_g = -1;
-    unsigned phase = 0, acc_phase = 0, qphase = 0;
-    bool ok = true;
-    while (c.left > 0) {
-      const int g = c.g;
-      if (g != prev_g) {
-        if (!mbar_wait(q_full, qphase, abort_flag)) { ok = false; break; }
-        qphase ^= 1u;
-        prev_g = g;
-      }
-      if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      TileCursor nx = c;
-      idx_cursor_next<RANGES>(nx, a, C::QG);
-      const bool last_of_group = (nx.left == 0) || (nx.g != g);
-      if (lane == 0) {
-        const unsigned d_tmem = tmem_base + acc * 256;
-        const uint64_t a0 = smem_desc_sw128(smem_u32(k_s + stage * C::K_TILE), 16, 1024);
-        const uint64_t b0 = smem_desc_sw128(smem_u32(q_s), 16, 1024);
+    } else {
+      // ---------------------------------------------------------- epilogue
+      while (e_ok && c.left > 0) {
+        const int g = c.g;
+        if (g != e_prev_g) {
+          if (!PILOT && !FB && e_prev_g >= 0) {
 #pragma unroll
-        for (int at = 0; at < C::ATOMS; ++at) {
+            for (int qq = 0; qq < QH; ++qq) flush(qq, e_prev_g);
+          }
+          // Each warp stages the head weights / thresholds of its own queries
+          // (no cross-warp barrier, so an aborting warp cannot strand the others).
+          __syncwarp();
+          if constexpr (QUAD) {
 #pragma unroll
-          for (int ks = 0; ks < C::KSTEPS_PER_ATOM; ++ks) {
-            // offsets go into the start-address field (address >> 4), which cannot carry
-            const uint64_t ad = a0 + static_cast<uint64_t>((at * C::BM * 128 + ks * 32) >> 4);
-            const uint64_t bd = b0 + static_cast<uint64_t>((at * C::BN * 128 + ks * 32) >> 4);
-            const unsigned accum = (at | ks) ? 1u : 0u;
-            if (FP8)
-              mma_fp8_ss(d_tmem, ad, bd, idesc, accum);
-            else
-              mma_bf16_ss(d_tmem, ad, bd, idesc, accum);
+            for (int qq = 0; qq < QH; ++qq) {
+              const int tl = g * C::QG + slot * QH + qq;
+#pragma unroll
+              for (int hp = 0; hp < HI / 8; ++hp) {
+                const long long o = static_cast<long long>(tl) * HI + 8 * hp + 2 * c4;
+                wreg[qq][hp] = (tl < a.Lb) ? make_float2(a.w[o], a.w[o + 1]) : make_float2(0.0f, 0.0f);
+              }
+            }
+          } else {
+            for (int j = lane; j < C::COLS; j += 32) {
+              const int tl = g * C::QG + slot * QH + j / HI;
+              w_w[j] = (tl < a.Lb) ? a.w[static_cast<long long>(g * C::QG + slot * QH) * HI + j] : 0.0f;
+            }
+          }
+          if (!PILOT && !FB) {
+            for (int j = lane; j < QH; j += 32) {
+              const int tl = g * C::QG + slot * QH + j;
+              tau_w[j] = (tl < a.Lb) ? threshold_float(a.tau[tl]) : INFINITY;
+              if (RANGES) {
+                lo_w[j] = (tl < a.Lb) ? a.key_lo[tl] : 0;
+                hi_w[j] = (tl < a.Lb) ? a.key_hi[tl] : 0;
+              }
+            }
+          }
+          __syncwarp();
+          e_prev_g = g;
+        }
+        if (!mbar_wait(&acc_full[e_acc], e_acc_phase, abort_flag)) { e_ok = false; break; }
+        tc_fence_after();
+        const unsigned taddr =
+            tmem_base + (static_cast<unsigned>(quarter * 32) << 16) + e_acc * 256 + slot * C::COLS;
+        // Score of (query qq of this warp, key): dense write (pilot), the
+        // fallback query's dense row, or threshold test and staging (main
+        // pass).  Called by all 32 lanes together.
+        auto emit = [&](int qq, int key, float score) {
+          const int tl = g * C::QG + slot * QH + qq;  // query within the block
+          if (PILOT) {
+            if (tl < a.Lb && key < a.n_keys) a.dense[static_cast<long long>(tl) * a.dense_ld + key] = score;
+          } else if (FB) {
+            if (tl == job_tl && key >= job_lo && key < job_hi)
+              a.dense[static_cast<long long>(blockIdx.x) * a.dense_ld + (key - job_lo)] = score;
+          } else {
+            const bool vis = RANGES ? (key >= lo_w[qq] && key < hi_w[qq]) : (key <= a.q_pos0 + tl);
+            const bool pass = (tl < a.Lb) && vis && (score >= tau_w[qq]);
+            const unsigned m = __ballot_sync(0xffffffffu, pass);
+            if (m) {
+              const int n = __popc(m);
+              if (cnt[qq] + n > SB) flush(qq, g);
+              if (pass) {
+                const unsigned long long k64 = (static_cast<unsigned long long>(float_order_key(score)) << 32) |
+                                               static_cast<unsigned>(~static_cast<unsigned>(key));
+                stg[qq * SB + cnt[qq] + __popc(m & lane_mask_lt)] = k64;
+              }
+              cnt[qq] += n;
+            }
+          }
+        };
+        if constexpr (QUAD) {
+          // 16-lane loads: this thread sees keys r4, r4 + 8, r4 + 16, r4 + 24 of the
+          // warp's 32 and, in every 8-column block, the two heads 2*c4, 2*c4 + 1.
+          // Its partial sums over those heads are added across the four threads
+          // of its quad; the thread ends with key r4 + 8*c4 for every query.
+          const int key = c.key0() + quarter * 32 + r4 + 8 * c4;
+          constexpr int NQ = 32 / HI;  // queries per 32-column chunk
+#pragma unroll
+          for (int ch = 0; ch < C::COLS / 32; ++ch) {
+            uint32_t va[16], vb[16];
+            tmem_ld_16x256b_x4(taddr + ch * 32, va);
+            tmem_ld_16x256b_x4(taddr + (16u << 16) + ch * 32, vb);
+            tmem_ld_wait();
+            if (ch == C::COLS / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&acc_empty[e_acc]);
+            }
+            float2 pa[NQ][4];
+#pragma unroll
+            for (int qc = 0; qc < NQ; ++qc)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) pa[qc][kk] = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int qc = (8 * j) / HI;
+              const float2 wv = wreg[ch * NQ + qc][((8 * j) % HI) / 8];
+              pa[qc][0] = ffma2(wv, relu2(va[4 * j], va[4 * j + 1]), pa[qc][0]);
+              pa[qc][1] = ffma2(wv, relu2(va[4 * j + 2], va[4 * j + 3]), pa[qc][1]);
+              pa[qc][2] = ffma2(wv, relu2(vb[4 * j], vb[4 * j + 1]), pa[qc][2]);
+              pa[qc][3] = ffma2(wv, relu2(vb[4 * j + 2], vb[4 * j + 3]), pa[qc][3]);
+            }
+#pragma unroll
+            for (int qc = 0; qc < NQ; ++qc) {
+              // Reduce-scatter over the quad: lane bit 1 picks keys {0,1} or {2,3},
+              // lane bit 0 one of the pair.  Every thread adds the same four
+              // partials in the same tree, ((p0 + p2) + (p1 + p3)).
+              const float v0 = pa[qc][0].x + pa[qc][0].y, v1 = pa[qc][1].x + pa[qc][1].y;
+              const float v2 = pa[qc][2].x + pa[qc][2].y, v3 = pa[qc][3].x + pa[qc][3].y;
+              const bool b1 = (c4 & 2) != 0, b0 = (c4 & 1) != 0;
+              float k0 = b1 ? v2 : v0, k1 = b1 ? v3 : v1;
+              k0 += __shfl_xor_sync(0xffffffffu, b1 ? v0 : v2, 2);
+              k1 += __shfl_xor_sync(0xffffffffu, b1 ? v1 : v3, 2);
+              float score = b0 ? k1 : k0;
+              score += __shfl_xor_sync(0xffffffffu, b0 ? k0 : k1, 1);
+              emit(ch * NQ + qc, key, score);
+            }
+          }
+        } else {
+          const int key = c.key0() + quarter * 32 + lane;
+          // One 32-column chunk of the accumulator at a time (keeps the live
+          // register set small); the buffer goes back to the MMA warp after the
+          // last chunk has been read.
+#pragma unroll
+          for (int ch = 0; ch < C::COLS / 32; ++ch) {
+            uint32_t vc[32];
+            tmem_ld_32x32b_x32(taddr + ch * 32, vc);
+            tmem_ld_wait();
+            if (ch == C::COLS / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&acc_empty[e_acc]);
+            }
+#pragma unroll
+            for (int qq = ch * 32 / HI; qq < (ch + 1) * 32 / HI; ++qq) {
+              const float4 *wq = reinterpret_cast<const float4 *>(w_w + qq * HI);
+              float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
+#pragma unroll
+              for (int h4 = 0; h4 < HI / 4; ++h4) {
+                const float4 w4 = wq[h4];
+                const int col = qq * HI + 4 * h4;
+                const float r0 = fmaxf(__uint_as_float(vc[(col + 0) % 32]), 0.0f);
+                const float r1 = fmaxf(__uint_as_float(vc[(col + 1) % 32]), 0.0f);
+                const float r2 = fmaxf(__uint_as_float(vc[(col + 2) % 32]), 0.0f);
+                const float r3 = fmaxf(__uint_as_float(vc[(col + 3) % 32]), 0.0f);
+                acc0 = ffma2(make_float2(w4.x, w4.y), make_float2(r0, r1), acc0);
+                acc1 = ffma2(make_float2(w4.z, w4.w), make_float2(r2, r3), acc1);
+              }
+              emit(qq, key, (acc0.x + acc1.x) + (acc0.y + acc1.y));
+            }
           }
         }
-        tc_commit(&empty[stage]);
-        tc_commit(&acc_full[acc]);
-        if (last_of_group) tc_commit(q_empty);
+        if (++e_acc == 2) { e_acc = 0; e_acc_phase ^= 1u; }
+        idx_cursor_next<RANGES>(c, a, C::QG);
       }
-      __syncwarp();
-      if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-      c = nx;
+      if (!e_ok) {
+        if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
+        *abort_flag = 1;
+      }
     }
-    if (!ok && lane == 0) {
-      atomicOr(a.status, DEV_TIMEOUT);
-      *abort_flag = 1;
+
+    if constexpr (FB) {
+      // The job's dense row is complete (every epilogue write precedes the
+      // barrier); the whole CTA selects its exact top-k from it.
+      __syncthreads();
+      if (!*abort_flag) {
+        const int need = min(a.topk, job_hi - job_lo);
+        DenseSelectSmem *sm = reinterpret_cast<DenseSelectSmem *>(smem + C::OFF_STG);
+        select_dense_row(a.dense + static_cast<long long>(blockIdx.x) * a.dense_ld, job_lo, job_hi - job_lo, need,
+                         a.topk, a.topk_idx + static_cast<long long>(job_tl) * a.topk,
+                         a.topk_score ? a.topk_score + static_cast<long long>(job_tl) * a.topk : nullptr, a.status,
+                         sm);
+      }
     }
+  }
+
+  if (warp == 0 && lane == 0) {
+    // Never leave with copies in flight.  Only the last STAGES issued tiles can
+    // still be landing, and each of them is the final use of its stage, so the
+    // phase parity below is unambiguous (an older phase of a reused stage would
+    // alias the current, never-completing one).
+    bool drained = true;
+    for (int i = (p_issued > C::STAGES ? p_issued - C::STAGES : 0); i < p_issued; ++i)
+      drained &= mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1u, nullptr);
+    if (p_q_issued > 0) drained &= mbar_wait(q_full, static_cast<unsigned>(p_q_issued - 1) & 1u, nullptr);
+    if (!drained) atomicOr(a.status, DEV_TIMEOUT);
+  } else if (warp == 1) {
     // Drain: every MMA this warp issued must finish before TMEM is released.
     if (lane == 0) {
       tc_commit(drain);
       if (!mbar_wait(drain, 0u, nullptr)) atomicOr(a.status, DEV_TIMEOUT);
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;          // 0..15
-    const int quarter = warp & 3;     // TMEM lane quarter this warp may access
-    const int slot = ew >> 2;         // which 64 accumulator columns
-    constexpr int QH = C::QH;         // queries per warp
-    constexpr int SB = C::SB;
-    TileCursor c = idx_cursor_begin<RANGES>(a, C::QG);
-    int acc = 0, prev_g = -1;
-    unsigned acc_phase = 0;
-    bool ok = true;
-    const unsigned lane_mask_lt = (1u << lane) - 1u;
-    float *w_w = w_s + ew * C::COLS;   // this warp's head weights: [QH queries][HI]
-    float *tau_w = tau_s + ew * C::COLS;
-    int *lo_w = reinterpret_cast<int *>(tau_w + QH);      // per-query key ranges (ranges mode)
-    int *hi_w = reinterpret_cast<int *>(tau_w + 2 * QH);
-    static_assert(3 * C::QH <= C::COLS, "thresholds and ranges share the per-warp slot");
-    unsigned long long *stg = reinterpret_cast<unsigned long long *>(smem + C::OFF_STG) + ew * QH * SB;
-    int cnt[QH];                   // staged candidates per query (warp-uniform)
-    // Indexer heads in whole 8-column blocks: 16-lane accumulator loads with the
-    // warp's head weights held in registers for the whole query group.
-    constexpr bool QUAD = (HI % 8) == 0;
-    const int c4 = lane & 3, r4 = lane >> 2;
-    float2 wreg[QH][HI / 8 > 0 ? HI / 8 : 1];
+  } else if (warp >= 2) {
+    if (e_ok && !PILOT && !FB && e_prev_g >= 0) {
 #pragma unroll
-    for (int qq = 0; qq < QH; ++qq) cnt[qq] = 0;
-
-    // Move a query's staged candidates to its global list: one atomic per batch.
-    auto flush = [&](int qq, int gq) {
-      const int n = cnt[qq];
-      if (n == 0) return;
-      const int tl = gq * C::QG + slot * QH + qq;
-      __syncwarp();
-      int base = 0;
-      if (lane == 0) base = atomicAdd(&a.cand_count[tl], n);
-      base = __shfl_sync(0xffffffffu, base, 0);
-      for (int i = lane; i < n; i += 32) {
-        const int pos = base + i;
-        if (pos < a.cap) a.cand[static_cast<long long>(tl) * a.cap + pos] = stg[qq * SB + i];
-      }
-      __syncwarp();
-      cnt[qq] = 0;
-    };
-
-    while (c.left > 0) {
-      const int g = c.g;
-      if (g != prev_g) {
-        if (!PILOT && prev_g >= 0) {
-#pragma unroll
-          for (int qq = 0; qq < QH; ++qq) flush(qq, prev_g);
-        }
-        // Each warp stages the head weights / thresholds of its own queries
-        // (no cross-warp barrier, so an aborting warp cannot strand the others).
-        __syncwarp();
-        if constexpr (QUAD) {
-#pragma unroll
-          for (int qq = 0; qq < QH; ++qq) {
-            const int tl = g * C::QG + slot * QH + qq;
-#pragma unroll
-            for (int hp = 0; hp < HI / 8; ++hp) {
-              const long long o = static_cast<long long>(tl) * HI + 8 * hp + 2 * c4;
-              wreg[qq][hp] = (tl < a.Lb) ? make_float2(a.w[o], a.w[o + 1]) : make_float2(0.0f, 0.0f);
-            }
-          }
-        } else {
-          for (int j = lane; j < C::COLS; j += 32) {
-            const int tl = g * C::QG + slot * QH + j / HI;
-            w_w[j] = (tl < a.Lb) ? a.w[static_cast<long long>(g * C::QG + slot * QH) * HI + j] : 0.0f;
-          }
-        }
-        if (!PILOT) {
-          for (int j = lane; j < QH; j += 32) {
-            const int tl = g * C::QG + slot * QH + j;
-            tau_w[j] = (tl < a.Lb) ? threshold_float(a.tau[tl]) : INFINITY;
-            if (RANGES) {
-              lo_w[j] = (tl < a.Lb) ? a.key_lo[tl] : 0;
-              hi_w[j] = (tl < a.Lb) ? a.key_hi[tl] : 0;
-            }
-          }
-        }
-        __syncwarp();
-        prev_g = g;
-      }
-      if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      const unsigned taddr =
-          tmem_base + (static_cast<unsigned>(quarter * 32) << 16) + acc * 256 + slot * C::COLS;
-      // Score of (query qq of this warp, key): dense write (pilot) or threshold
-      // test and staging (main pass).  Called by all 32 lanes together.
-      auto emit = [&](int qq, int key, float score) {
-        const int tl = g * C::QG + slot * QH + qq;  // query within the block
-        if (PILOT) {
-          if (tl < a.Lb && key < a.n_keys) a.dense[static_cast<long long>(tl) * a.dense_ld + key] = score;
-        } else {
-          const bool vis = RANGES ? (key >= lo_w[qq] && key < hi_w[qq]) : (key <= a.q_pos0 + tl);
-          const bool pass = (tl < a.Lb) && vis && (score >= tau_w[qq]);
-          const unsigned m = __ballot_sync(0xffffffffu, pass);
-          if (m) {
-            const int n = __popc(m);
-            if (cnt[qq] + n > SB) flush(qq, g);
-            if (pass) {
-              const unsigned long long k64 = (static_cast<unsigned long long>(float_order_key(score)) << 32) |
-                                             static_cast<unsigned>(~static_cast<unsigned>(key));
-              stg[qq * SB + cnt[qq] + __popc(m & lane_mask_lt)] = k64;
-            }
-            cnt[qq] += n;
-          }
-        }
-      };
-      if constexpr (QUAD) {
-        // 16-lane loads: this thread sees keys r4, r4 + 8, r4 + 16, r4 + 24 of the
-        // warp's 32 and, in every 8-column block, the two heads 2*c4, 2*c4 + 1.
-        // Its partial sums over those heads are added across the four threads
-        // of its quad; the thread ends with key r4 + 8*c4 for every query.
-        const int key = c.key0() + quarter * 32 + r4 + 8 * c4;
-        constexpr int NQ = 32 / HI;  // queries per 32-column chunk
-#pragma unroll
-        for (int ch = 0; ch < C::COLS / 32; ++ch) {
-          uint32_t va[16], vb[16];
-          tmem_ld_16x256b_x4(taddr + ch * 32, va);
-          tmem_ld_16x256b_x4(taddr + (16u << 16) + ch * 32, vb);
-          tmem_ld_wait();
-          if (ch == C::COLS / 32 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
-          }
-          float2 pa[NQ][4];
-#pragma unroll
-          for (int qc = 0; qc < NQ; ++qc)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) pa[qc][kk] = make_float2(0.0f, 0.0f);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int qc = (8 * j) / HI;
-            const float2 wv = wreg[ch * NQ + qc][((8 * j) % HI) / 8];
-            pa[qc][0] = ffma2(wv, relu2(va[4 * j], va[4 * j + 1]), pa[qc][0]);
-            pa[qc][1] = ffma2(wv, relu2(va[4 * j + 2], va[4 * j + 3]), pa[qc][1]);
-            pa[qc][2] = ffma2(wv, relu2(vb[4 * j], vb[4 * j + 1]), pa[qc][2]);
-            pa[qc][3] = ffma2(wv, relu2(vb[4 * j + 2], vb[4 * j + 3]), pa[qc][3]);
-          }
-#pragma unroll
-          for (int qc = 0; qc < NQ; ++qc) {
-            // Reduce-scatter over the quad: lane bit 1 picks keys {0,1} or {2,3},
-            // lane bit 0 one of the pair.  Every thread adds the same four
-            // partials in the same tree, ((p0 + p2) + (p1 + p3)).
-            const float v0 = pa[qc][0].x + pa[qc][0].y, v1 = pa[qc][1].x + pa[qc][1].y;
-            const float v2 = pa[qc][2].x + pa[qc][2].y, v3 = pa[qc][3].x + pa[qc][3].y;
-            const bool b1 = (c4 & 2) != 0, b0 = (c4 & 1) != 0;
-            float k0 = b1 ? v2 : v0, k1 = b1 ? v3 : v1;
-            k0 += __shfl_xor_sync(0xffffffffu, b1 ? v0 : v2, 2);
-            k1 += __shfl_xor_sync(0xffffffffu, b1 ? v1 : v3, 2);
-            float score = b0 ? k1 : k0;
-            score += __shfl_xor_sync(0xffffffffu, b0 ? k0 : k1, 1);
-            emit(ch * NQ + qc, key, score);
-          }
-        }
-      } else {
-        const int key = c.key0() + quarter * 32 + lane;
-        // One 32-column chunk of the accumulator at a time (keeps the live
-        // register set small); the buffer goes back to the MMA warp after the
-        // last chunk has been read.
-#pragma unroll
-        for (int ch = 0; ch < C::COLS / 32; ++ch) {
-          uint32_t vc[32];
-          tmem_ld_32x32b_x32(taddr + ch * 32, vc);
-          tmem_ld_wait();
-          if (ch == C::COLS / 32 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
-          }
-#pragma unroll
-          for (int qq = ch * 32 / HI; qq < (ch + 1) * 32 / HI; ++qq) {
-            const float4 *wq = reinterpret_cast<const float4 *>(w_w + qq * HI);
-            float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
-#pragma unroll
-            for (int h4 = 0; h4 < HI / 4; ++h4) {
-              const float4 w4 = wq[h4];
-              const int col = qq * HI + 4 * h4;
-              const float r0 = fmaxf(__uint_as_float(vc[(col + 0) % 32]), 0.0f);
-              const float r1 = fmaxf(__uint_as_float(vc[(col + 1) % 32]), 0.0f);
-              const float r2 = fmaxf(__uint_as_float(vc[(col + 2) % 32]), 0.0f);
-              const float r3 = fmaxf(__uint_as_float(vc[(col + 3) % 32]), 0.0f);
-              acc0 = ffma2(make_float2(w4.x, w4.y), make_float2(r0, r1), acc0);
-              acc1 = ffma2(make_float2(w4.z, w4.w), make_float2(r2, r3), acc1);
-            }
-            emit(qq, key, (acc0.x + acc1.x) + (acc0.y + acc1.y));
-          }
-        }
-      }
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-      idx_cursor_next<RANGES>(c, a, C::QG);
-    }
-    if (ok && !PILOT && prev_g >= 0) {
-#pragma unroll
-      for (int qq = 0; qq < QH; ++qq) flush(qq, prev_g);
-    }
-    if (!ok) {
-      if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
-      *abort_flag = 1;
+      for (int qq = 0; qq < QH; ++qq) flush(qq, e_prev_g);
     }
   }
 
@@ -542,11 +615,11 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
   }
 }
 
-template <int DI, int HI, bool FP8, bool PILOT, bool RANGES>
+template <int DI, int HI, bool FP8, int MODE, bool RANGES>
 static cudaError_t launch_indexer_t(const CUtensorMap &tq, const CUtensorMap &tk, const IndexerArgs &a, int grid,
                                     cudaStream_t stream) {
   using C = IdxCfg<DI, HI, FP8>;
-  auto kern = indexer_kernel<DI, HI, FP8, PILOT, RANGES>;
+  auto kern = indexer_kernel<DI, HI, FP8, MODE, RANGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   return launch_kernel(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream, tq, tk, a);
@@ -554,13 +627,26 @@ static cudaError_t launch_indexer_t(const CUtensorMap &tq, const CUtensorMap &tk
 
 int indexer_queries_per_group(int H_I) { return 256 / H_I; }
 
+template <int DI, int HI, bool FP8>
+static cudaError_t launch_indexer_mode(const CUtensorMap &tq, const CUtensorMap &tk, const IndexerArgs &a,
+                                       IndexerMode mode, int grid, cudaStream_t stream) {
+  const bool ranges = a.key_lo != nullptr;
+  switch (mode) {
+    case kIdxPilot: return launch_indexer_t<DI, HI, FP8, kIdxPilot, false>(tq, tk, a, grid, stream);
+    case kIdxEmit:
+      return ranges ? launch_indexer_t<DI, HI, FP8, kIdxEmit, true>(tq, tk, a, grid, stream)
+                    : launch_indexer_t<DI, HI, FP8, kIdxEmit, false>(tq, tk, a, grid, stream);
+    case kIdxFallback:
+      return ranges ? launch_indexer_t<DI, HI, FP8, kIdxFallback, true>(tq, tk, a, grid, stream)
+                    : launch_indexer_t<DI, HI, FP8, kIdxFallback, false>(tq, tk, a, grid, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_indexer(const CUtensorMap &tq, const CUtensorMap &tk, const IndexerArgs &a, int D_I, int H_I,
-                           bool fp8, bool pilot, int grid, cudaStream_t stream) {
-#define DSA_IDX_CASE(DI_, HI_, FP8_)                                                            \
-  if (D_I == DI_ && H_I == HI_ && fp8 == FP8_)                                                  \
-    return pilot            ? launch_indexer_t<DI_, HI_, FP8_, true, false>(tq, tk, a, grid, stream)  \
-           : a.key_lo != nullptr ? launch_indexer_t<DI_, HI_, FP8_, false, true>(tq, tk, a, grid, stream) \
-                             : launch_indexer_t<DI_, HI_, FP8_, false, false>(tq, tk, a, grid, stream);
+                           bool fp8, IndexerMode mode, int grid, cudaStream_t stream) {
+#define DSA_IDX_CASE(DI_, HI_, FP8_) \
+  if (D_I == DI_ && H_I == HI_ && fp8 == FP8_) return launch_indexer_mode<DI_, HI_, FP8_>(tq, tk, a, mode, grid, stream);
   DSA_IDX_CASE(128, 32, false)
   DSA_IDX_CASE(128, 32, true)
   DSA_IDX_CASE(64, 4, false)

@@ -15,77 +15,23 @@
 //      k-th best; the winners are emitted in ascending key order with -1
 //      padding (the int32 index-mask convention of llama.cpp PR #25917,
 //      discussion).  Equal scores go to the smaller index.
-//   3. fallback_kernel: any query the sample misjudged (too few or too many
-//      candidates) is rescored over all visible keys on the CUDA cores and
-//      selected exactly, so the result never depends on the sample.
-#include <cuda_fp8.h>
+//   3. the exact fallback: any query the sample misjudged (too few or too
+//      many candidates) is rescored over all its visible keys by the indexer
+//      kernel itself (FALLBACK mode, indexer.cu), with the same tensor-core
+//      arithmetic as the main pass, and selected exactly from the dense row;
+//      so neither the sample nor the query blocking can change a selection.
 #include <cuda_runtime.h>
 
 #include <cmath>
 
 #include "dsa_internal.h"
 #include "ptx.cuh"
+#include "select_common.cuh"
 
 namespace dsa {
 
 constexpr int kSelThreads = 512;
 constexpr int kMaxTopk = 4096;
-
-// Block-wide MSB-first radix select.  Among n unique keys (fetch(i), i < n) find
-// (prefix, mask) such that exactly `need` keys satisfy (key & mask) >= prefix,
-// i.e. key >= prefix.  1 <= need <= n.  Every thread of the block must call it.
-template <typename KeyT, typename Fetch>
-__device__ void block_radix_select(Fetch fetch, int n, int need, KeyT &prefix_out, KeyT &mask_out,
-                                   unsigned *hist, unsigned *misc) {
-  constexpr int BITS = sizeof(KeyT) * 8;
-  KeyT prefix = 0, mask = 0;
-  unsigned remaining = static_cast<unsigned>(need);
-  for (int shift = BITS - 8; shift >= 0; shift -= 8) {
-    for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[b] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const KeyT k = fetch(i);
-      if ((k & mask) == prefix) atomicAdd(&hist[static_cast<unsigned>(k >> shift) & 255u], 1u);
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      const int lane = threadIdx.x;
-      unsigned local = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) local += hist[255 - 8 * lane - j];
-      unsigned incl = local;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-      }
-      const unsigned excl = incl - local;
-      if (excl < remaining && remaining <= incl) {
-        unsigned c = excl;
-        for (int j = 0; j < 8; ++j) {
-          const int bin = 255 - 8 * lane - j;
-          if (c + hist[bin] >= remaining) {
-            misc[0] = static_cast<unsigned>(bin);
-            misc[1] = remaining - c;
-            misc[2] = hist[bin];
-            break;
-          }
-          c += hist[bin];
-        }
-      }
-    }
-    __syncthreads();
-    const unsigned chosen = misc[0];
-    remaining = misc[1];
-    const unsigned cnt = misc[2];
-    prefix |= static_cast<KeyT>(chosen) << shift;
-    mask |= static_cast<KeyT>(0xFF) << shift;
-    __syncthreads();
-    if (cnt == remaining) break;
-  }
-  prefix_out = prefix;
-  mask_out = mask;
-}
 
 // ------------------------------------------------------------------ threshold
 constexpr int kMaxSamples = 4096;
@@ -156,32 +102,6 @@ __device__ void block_bitonic_sort(unsigned long long *v, int n) {
 constexpr int kSmemCand = 8192;        // candidates staged in shared memory (larger lists stay in L2)
 constexpr int kBitmapKeys = 262144;    // ascending output through a shared bitmap up to this many keys
 
-// Exclusive prefix sum of one int per thread over the block (blockDim.x <= 1024).
-__device__ int block_exclusive_scan(int v, int *warp_tot, int *total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = (blockDim.x + 31) >> 5;
-  int incl = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += o;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int t = lane < nwarps ? warp_tot[lane] : 0;
-    int ti = t;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, ti, off);
-      if (lane >= off) ti += o;
-    }
-    if (lane < nwarps) warp_tot[lane] = ti - t;
-    if (lane == 31) *total = ti;
-  }
-  __syncthreads();
-  return warp_tot[warp] + incl - v;
-}
-
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   pdl_wait_and_release();
   extern __shared__ __align__(16) unsigned char sel_smem[];
@@ -197,7 +117,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   const int nvis = a.key_lo != nullptr ? a.key_hi[tl] - lo : a.q_pos0 + tl + 1;
   const int need = min(a.topk, nvis);
   const int count = a.cand_count[tl];
-  if (count > a.cap || count < need) {
+  const bool fallback = count > a.cap || count < need;
+  if (threadIdx.x == 0 && a.stats != nullptr) {
+    atomicAdd(&a.stats->candidates, static_cast<unsigned long long>(count));
+    atomicAdd(&a.stats->queries, 1u);
+    atomicMax(&a.stats->max_candidates, static_cast<unsigned>(count));
+    if (fallback) atomicAdd(&a.stats->fallback_queries, 1u);
+  }
+  if (fallback) {
     if (threadIdx.x == 0) {
       const int pos = atomicAdd(&a.fb_counters[0], 1);
       a.fb_list[pos] = tl;
@@ -275,101 +202,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
       out[j] = static_cast<int32_t>(v >> 32);
       if (osc) osc[j] = order_key_float(static_cast<unsigned>(v & 0xFFFFFFFFull));
     } else {
-      out[j] = -1;
-      if (osc) osc[j] = -INFINITY;
-    }
-  }
-}
-
-// ------------------------------------------------------------------ fallback
-__device__ __forceinline__ float idx_elem(const void *base, long long i, int fp8) {
-  if (fp8) {
-    const __nv_fp8_storage_t b = static_cast<const unsigned char *>(base)[i];
-    return __half2float(__half(__nv_cvt_fp8_to_halfraw(b, __NV_E4M3)));
-  }
-  const unsigned short b = static_cast<const unsigned short *>(base)[i];
-  return __uint_as_float(static_cast<unsigned>(b) << 16);
-}
-
-__global__ void __launch_bounds__(kSelThreads) fallback_kernel(SelectArgs a) {
-  pdl_wait_and_release();
-  extern __shared__ float fb_smem[];
-  __shared__ unsigned hist[256];
-  __shared__ unsigned misc[4];
-  __shared__ int job;
-  __shared__ int warp_cnt[kSelThreads / 32];
-  __shared__ int warp_off[kSelThreads / 32];
-  __shared__ int base_s;
-  float *q_s = fb_smem;                       // [H_I][D_I]
-  float *w_s = fb_smem + a.H_I * a.D_I;        // [H_I]
-  float *scores = a.fb_scratch + static_cast<long long>(blockIdx.x) * a.N;
-  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
-  while (true) {
-    __syncthreads();
-    if (threadIdx.x == 0) job = atomicAdd(&a.fb_counters[1], 1);
-    __syncthreads();
-    if (job >= *reinterpret_cast<volatile int *>(&a.fb_counters[0])) break;
-    const int tl = a.fb_list[job];
-    const int t = a.t0 + tl;
-    const int lo = a.key_lo != nullptr ? a.key_lo[tl] : 0;  // visible keys [lo, lo + nvis)
-    const int nvis = a.key_lo != nullptr ? a.key_hi[tl] - lo : a.q_pos0 + tl + 1;
-    const int need = min(a.topk, nvis);
-    for (int i = threadIdx.x; i < a.H_I * a.D_I; i += blockDim.x)
-      q_s[i] = idx_elem(a.q_idx, static_cast<long long>(t) * a.H_I * a.D_I + i, a.fp8);
-    for (int i = threadIdx.x; i < a.H_I; i += blockDim.x) w_s[i] = a.w[static_cast<long long>(t) * a.H_I + i];
-    __syncthreads();
-    for (int j = threadIdx.x; j < nvis; j += blockDim.x) {
-      const int s = lo + j;
-      float kr[128];
-      for (int d = 0; d < a.D_I; ++d) kr[d] = idx_elem(a.k_idx, static_cast<long long>(s) * a.ldk + d, a.fp8);
-      float score = 0.0f;
-      for (int h = 0; h < a.H_I; ++h) {
-        float dot = 0.0f;
-        for (int d = 0; d < a.D_I; ++d) dot = fmaf(q_s[h * a.D_I + d], kr[d], dot);
-        score = fmaf(w_s[h], fmaxf(dot, 0.0f), score);
-      }
-      scores[j] = score;
-    }
-    __syncthreads();
-    // j indexes the visible keys; key lo + j breaks ties
-    auto key_of = [&](int j) {
-      return (static_cast<unsigned long long>(float_order_key(scores[j])) << 32) |
-             static_cast<unsigned>(~static_cast<unsigned>(lo + j));
-    };
-    unsigned long long prefix = 0, mask = 0;
-    if (nvis > need) block_radix_select<unsigned long long>(key_of, nvis, need, prefix, mask, hist, misc);
-    if (threadIdx.x == 0) base_s = 0;
-    __syncthreads();
-    int32_t *out = a.topk_idx + static_cast<long long>(t) * a.topk;
-    float *osc = a.topk_score ? a.topk_score + static_cast<long long>(t) * a.topk : nullptr;
-    for (int s0 = 0; s0 < nvis; s0 += blockDim.x) {
-      const int s = s0 + threadIdx.x;
-      const bool sel = (s < nvis) && (key_of(min(s, nvis - 1)) >= prefix);
-      const unsigned bal = __ballot_sync(0xffffffffu, sel);
-      if (lane == 0) warp_cnt[warp] = __popc(bal);
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int w = 0; w < kSelThreads / 32; ++w) {
-          warp_off[w] = acc;
-          acc += warp_cnt[w];
-        }
-        misc[3] = static_cast<unsigned>(acc);
-      }
-      __syncthreads();
-      if (sel) {
-        const int pos = base_s + warp_off[warp] + __popc(bal & ((1u << lane) - 1u));
-        if (pos < need) {
-          out[pos] = lo + s;
-          if (osc) osc[pos] = scores[s];
-        }
-      }
-      __syncthreads();
-      if (threadIdx.x == 0) base_s += static_cast<int>(misc[3]);
-      __syncthreads();
-    }
-    if (threadIdx.x == 0 && base_s != need) atomicOr(a.status, DEV_OVERFLOW);
-    for (int j = need + threadIdx.x; j < a.topk; j += blockDim.x) {
       out[j] = -1;
       if (osc) osc[j] = -INFINITY;
     }
@@ -561,9 +393,5 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream) {
   return launch_kernel(select_kernel, dim3(a.Lb), dim3(kSelThreads), smem, stream, a);
 }
 
-cudaError_t launch_fallback(const SelectArgs &a, cudaStream_t stream) {
-  const int smem = (a.H_I * a.D_I + a.H_I) * static_cast<int>(sizeof(float));
-  return launch_kernel(fallback_kernel, dim3(a.fb_slots), dim3(kSelThreads), smem, stream, a);
-}
 
 }  // namespace dsa

@@ -22,8 +22,13 @@ q in blocks of 64 query rows so that peak host memory stays bounded):
 * ``concentrated``: N(0, 1) plus a shared mean direction mu = 2 * u, u a
   seeded uniform unit vector in R^D_I, added to every q_idx head row and every
   k_idx row, then rounded to e4m3 (RNE, saturated to +-448);
+* ``walk`` (a stress input with correlated neighbouring queries, not one of
+  the five workloads): k_idx N(0, 1); q_idx[0] N(0, 1) and q_idx[t] =
+  q_idx[t-1] + 0.05 N(0, 1) elementwise, so neighbouring queries select
+  mostly the same keys; rounded to bf16;
 * weights ``normal_half`` N(0,1)/2, ``int12`` integers in {1, 2},
-  ``normal_rsqrt`` N(0,1)/sqrt(H_I);
+  ``normal_rsqrt`` N(0,1)/sqrt(H_I), ``walk_rsqrt``: w[0] N(0,1)/sqrt(H_I) and
+  w[t] = w[t-1] + 0.05 N(0,1)/sqrt(H_I);
 * MLA latent and rope columns N(0, std^2) with the stated standard deviations.
 """
 from __future__ import annotations
@@ -48,8 +53,8 @@ class ChunkConfig:
     H_I: int
     D_I: int
     idx_dtype: str  # "bf16" | "e4m3"
-    idx_dist: str  # "normal" | "int3" | "concentrated"
-    w_dist: str  # "normal_half" | "int12" | "normal_rsqrt"
+    idx_dist: str  # "normal" | "int3" | "concentrated" | "walk"
+    w_dist: str  # "normal_half" | "int12" | "normal_rsqrt" | "walk_rsqrt"
     topk: int
     H: int
     lat_std: float
@@ -91,7 +96,12 @@ WORKLOADS = [TINY, TIES, CTX64K, CTX128K, CTX256K]
 DECODE128K = ChunkConfig("dsa-decode-128k-N131072-L1", N=131072, L=1, H_I=32, D_I=128, idx_dtype="bf16",
                          idx_dist="normal", w_dist="normal_rsqrt", topk=2048, H=64, lat_std=0.5, rope_std=0.5,
                          seed=3)
-BY_NAME = {c.name: c for c in WORKLOADS + [DECODE128K]}
+# Stress input for candidate-overlap reuse: queries whose selections overlap
+# heavily (q_idx and w random walks over the queries).  Not a benchmark workload.
+CORRELATED = ChunkConfig("dsa-correlated-N65536-L1024", N=65536, L=1024, H_I=32, D_I=128, idx_dtype="bf16",
+                         idx_dist="walk", w_dist="walk_rsqrt", topk=2048, H=64, lat_std=0.5, rope_std=0.5, seed=5)
+WALK_STEP = 0.05
+BY_NAME = {c.name: c for c in WORKLOADS + [DECODE128K, CORRELATED]}
 
 
 def small_variant(cfg: ChunkConfig, N: int, L: int, topk: int | None = None, H: int | None = None,
@@ -107,12 +117,15 @@ def _to_idx_storage(x: torch.Tensor, dtype: str) -> torch.Tensor:
     return x.clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
 
 
-def _draw_idx(g: torch.Generator, shape, dist: str, mu: torch.Tensor | None) -> torch.Tensor:
+def _draw_idx(g: torch.Generator, shape, dist: str, mu: torch.Tensor | None, walk: bool = False) -> torch.Tensor:
     if dist == "int3":
         return torch.randint(-3, 4, shape, generator=g).to(torch.float32)
     x = torch.randn(shape, generator=g, dtype=torch.float32)
     if dist == "concentrated":
         x += mu
+    if dist == "walk" and walk:  # along the first axis: x[t] = x[t-1] + WALK_STEP * N(0, 1)
+        x[1:] *= WALK_STEP
+        x = torch.cumsum(x, dim=0)
     return x
 
 
@@ -135,13 +148,17 @@ def generate(cfg: ChunkConfig, with_mla: bool = True) -> dict:
         u = torch.randn(cfg.D_I, generator=g, dtype=torch.float64)
         mu = (2.0 * u / u.norm()).to(torch.float32)
     k_idx = _to_idx_storage(_draw_idx(g, (cfg.N, cfg.D_I), cfg.idx_dist, mu), cfg.idx_dtype)
-    q_idx = _to_idx_storage(_draw_idx(g, (cfg.L, cfg.H_I, cfg.D_I), cfg.idx_dist, mu), cfg.idx_dtype)
+    q_idx = _to_idx_storage(_draw_idx(g, (cfg.L, cfg.H_I, cfg.D_I), cfg.idx_dist, mu, walk=True), cfg.idx_dtype)
     if cfg.w_dist == "int12":
         w = torch.randint(1, 3, (cfg.L, cfg.H_I), generator=g).to(torch.float32)
     elif cfg.w_dist == "normal_half":
         w = torch.randn(cfg.L, cfg.H_I, generator=g, dtype=torch.float32) / 2.0
     elif cfg.w_dist == "normal_rsqrt":
         w = torch.randn(cfg.L, cfg.H_I, generator=g, dtype=torch.float32) / math.sqrt(cfg.H_I)
+    elif cfg.w_dist == "walk_rsqrt":
+        w = torch.randn(cfg.L, cfg.H_I, generator=g, dtype=torch.float32)
+        w[1:] *= WALK_STEP
+        w = torch.cumsum(w, dim=0) / math.sqrt(cfg.H_I)
     else:
         raise ValueError(cfg.w_dist)
     out = {"q_idx": q_idx.contiguous(), "k_idx": k_idx.contiguous(), "w": w.contiguous()}

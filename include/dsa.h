@@ -39,7 +39,10 @@
  *     are returned before anything is launched; a failed launch returns
  *     DSA_ERR_CUDA.  Device-side conditions (a wait that timed out, an
  *     out-of-range index) are recorded in the workspace's status word and read
- *     back with dsa_workspace_status().
+ *     back with dsa_workspace_status(), which plays the role of an explicit
+ *     check: every entry point clears the word when it starts (it never
+ *     synchronises to look at the previous call's word), so read it after a
+ *     call and before the next call on the same workspace.
  *   - No function aborts the process or throws across the ABI.
  */
 #ifndef DSA_H_
@@ -105,34 +108,15 @@ size_t dsa_indexer_topk_workspace(int L, int N, int H_I, int D_I, int topk, dsa_
  * Supported: D_I = 128 with H_I in {8, 16, 32} (bf16 or fp8), D_I = 64 with
  * H_I in {4, 32} (bf16); 1 <= topk <= 4096.  Queries are processed in blocks of
  * up to 1,024 (mlx-lm PR #1997, "How it works": long chunks split into query
- * blocks); the result does not depend on the blocking.
+ * blocks); the result does not depend on the blocking: every score is computed
+ * by the same tensor-core instruction sequence wherever the query falls, the
+ * queries the threshold sample misjudges included.
  */
 dsa_status_t dsa_indexer_topk(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
                               dsa_dtype_t dtype, int L, int N, int H_I, int D_I, int q_pos0, int topk,
                               int32_t *topk_idx, float *topk_score, void *workspace, size_t workspace_bytes,
                               dsa_stream_t stream);
 
-/*
- * dsa_indexer_topk for callers that cannot allocate device memory: code that
- * runs inside a CUDA graph being captured or replayed, code that owns no
- * allocator (an inference runtime whose memory is planned once up front), or
- * a process whose device memory is already fully reserved.  Same arguments
- * and results as dsa_indexer_topk, minus the workspace: the scratch is one
- * fixed 16 MiB device array inside libdsa.so (every GPU that loads the library
- * holds it until the process exits).  The pages describe no counterpart; this
- * is a property of this library only.
- *
- *   - Limit: problems whose scratch exceeds 16 MiB at 64-query blocks are
- *     rejected with DSA_ERR_WORKSPACE before anything is launched (with
- *     top-k <= 2048 that admits N up to about 180,000 cached keys).
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
- *   - No cudaMalloc or cudaFree, and no allocating library call, is made.
- *   - Every call on a device shares the one array, which keeps the previous
- *     call's contents; the call clears what must start at zero.  Calls that
- *     overlap on the GPU (two streams, two host threads) race on the array
- *     and must be serialised by the caller.
- */
 /*
  * dsa_indexer_topk with general visibility carried by an index mask instead of
  * the causal triangle (llama.cpp PR #25917, discussion: causality applied to
@@ -156,9 +140,44 @@ dsa_status_t dsa_indexer_topk_ranges(const void *q_idx, const void *k_idx, int64
                                      const int32_t *key_hi, int topk, int32_t *topk_idx, float *topk_score,
                                      void *workspace, size_t workspace_bytes, dsa_stream_t stream);
 
+/*
+ * dsa_indexer_topk for callers that cannot allocate device memory: code that
+ * owns no allocator (an inference runtime whose memory is planned once up
+ * front and hands kernels only their inputs and outputs), or a process whose
+ * device memory is already fully reserved by others.  Same arguments and
+ * results as dsa_indexer_topk, minus the workspace: the scratch is one fixed
+ * 16 MiB device array inside libdsa.so (every GPU that loads the library holds
+ * it until the process exits).  The pages describe no counterpart; this is a
+ * property of this library only.
+ *
+ *   - Limit: problems whose scratch exceeds 16 MiB at 64-query blocks are
+ *     rejected with DSA_ERR_WORKSPACE before anything is launched (with
+ *     top-k <= 2048 that admits N up to about 180,000 cached keys).
+ *   - The first call on each device (each CUDA context: again after a device
+ *     reset) looks up the array's device address with cudaGetSymbolAddress;
+ *     make that first call before any stream capture.
+ *   - No cudaMalloc or cudaFree, and no allocating library call, is made.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents; the call clears what must start at zero.  Calls that
+ *     overlap on the GPU (two streams, two host threads) race on the array
+ *     and must be serialised by the caller.
+ *   - Device-side conditions land in the array's status word; read them with
+ *     dsa_indexer_topk_noalloc_status.
+ */
 dsa_status_t dsa_indexer_topk_noalloc(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
                                       dsa_dtype_t dtype, int L, int N, int H_I, int D_I, int q_pos0, int topk,
                                       int32_t *topk_idx, float *topk_score, dsa_stream_t stream);
+
+/*
+ * Status of the fixed scratch of dsa_indexer_topk_noalloc on the current
+ * device: synchronises `stream`, reads the array's status word (bits as in
+ * dsa_workspace_status) into *flags and returns DSA_OK when it is zero,
+ * DSA_ERR_INTERNAL when it is not, DSA_ERR_CUDA on a CUDA error.  Like the
+ * workspace's word, it describes the most recent dsa_indexer_topk_noalloc call
+ * on the device, which clears it when it starts.  The pages have no
+ * counterpart.
+ */
+dsa_status_t dsa_indexer_topk_noalloc_status(dsa_stream_t stream, unsigned *flags);
 
 /* Workspace (bytes) for dsa_sparse_mla_prefill: the status word, plus the
  * union buffers of packed attention (H <= 32) or the fp32 partial results of
@@ -200,13 +219,15 @@ dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, int64_t ldkv,
                                     size_t workspace_bytes, dsa_stream_t stream);
 
 /* Workspace (bytes) for dsa_prefill_chunk with these sizes (query_block <= 0
- * selects 1,024). */
+ * selects 1,024; rounded up as dsa_prefill_chunk does). */
 size_t dsa_prefill_chunk_workspace(int L, int N, int H_I, int D_I, int H, int topk, int query_block,
                                    dsa_dtype_t dtype, int want_topk_out);
 
 /*
  * All three stages for one prefill chunk, query block by query block
- * (query_block <= 0 selects 1,024 queries per block).
+ * (query_block <= 0 selects 1,024 queries per block; a block size is rounded
+ * up to a whole number of the indexer's query groups, 256 / H_I queries, e.g.
+ * 8 at H_I = 32).  Selections and outputs are bit-identical for every blocking.
  *
  *   q_idx, k_idx, ldk, w, dtype, H_I, D_I : as dsa_indexer_topk
  *   q, kv, ldkv, H, scale                 : as dsa_sparse_mla_prefill
@@ -267,9 +288,29 @@ dsa_status_t dsa_selftest_wait_timeout(void *workspace, size_t workspace_bytes, 
  * timed out, bit 1: an index outside [0, N) reached the attention stage,
  * bit 2: an internal selection count mismatch).  Returns DSA_OK when the word
  * is zero, DSA_ERR_INTERNAL when it is not, DSA_ERR_CUDA on a CUDA error.
- * Every entry point clears the word when it starts.
+ * Every entry point clears the word when it starts, so the word describes the
+ * most recent call on this workspace: this is the explicit check of that call.
  */
 dsa_status_t dsa_workspace_status(const void *workspace, dsa_stream_t stream, unsigned *flags);
+
+/* Selection totals of the most recent dsa_indexer_topk* / dsa_prefill_chunk*
+ * call on a workspace, over all its query blocks (cleared when a call starts). */
+typedef struct {
+  unsigned long long candidates; /* candidate keys written back (above the sample threshold), all queries */
+  unsigned queries;              /* queries selected */
+  unsigned fallback_queries;     /* queries the threshold sample misjudged, resolved by the exact fallback */
+  unsigned max_candidates;       /* largest candidate count of one query */
+  unsigned reserved;
+} dsa_selection_stats_t;
+
+/*
+ * Diagnostic with no counterpart in the method: synchronise `stream` and copy
+ * the selection totals above from `workspace` (DSA_ERR_INVALID_ARG for NULL
+ * pointers, DSA_ERR_CUDA on a CUDA error).  LiteTopK (arXiv 2607.11976,
+ * Abstract) writes back only promising candidates; these totals show how many.
+ */
+dsa_status_t dsa_workspace_selection_stats(const void *workspace, dsa_stream_t stream,
+                                           dsa_selection_stats_t *stats);
 
 #ifdef __cplusplus
 }

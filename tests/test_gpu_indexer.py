@@ -125,3 +125,7 @@ def test_supported_indexer_shapes(D_I, H_I, fp8):
     assert tuple(inp["q_idx"].shape) == (cfg.L, H_I, D_I)
     idx, sc = run_indexer(cfg, inp, with_scores=True)
     check_rows(cfg, inp, idx, list(range(0, cfg.L, 7)) + [cfg.L - 1], gpu_scores=sc)
+    # the exact fallback (candidate capacity 64 < top-k: every query) scores with the same arithmetic
+    full = dsa.dsa_indexer_topk_workspace(cfg.L, cfg.N, cfg.H_I, cfg.D_I, cfg.topk)
+    idx_f, sc_f = run_indexer(cfg, inp, ws_bytes=full - cfg.L * (8192 - 64) * 8, with_scores=True)
+    assert np.array_equal(idx, idx_f) and np.array_equal(sc, sc_f)

@@ -15,14 +15,17 @@ REL_L2 = 1e-2
 MAX_ABS = 3e-2
 
 
-def run_ranges(cfg, inp, lo, hi):
+def run_ranges(cfg, inp, lo, hi, ws_bytes=None, with_scores=False):
     dev = torch.device("cuda")
     g = {k: v.to(dev) for k, v in inp.items()}
     idx = torch.full((cfg.L, cfg.topk), -7, dtype=torch.int32, device=dev)
-    ws = dsa.alloc_workspace(dsa.dsa_indexer_topk_workspace(cfg.L, cfg.N, cfg.H_I, cfg.D_I, cfg.topk,
-                                                            dsa._dtype_code(g["q_idx"])), dev)
+    sc = torch.full((cfg.L, cfg.topk), float("nan"), dtype=torch.float32, device=dev) if with_scores else None
+    full = dsa.dsa_indexer_topk_workspace(cfg.L, cfg.N, cfg.H_I, cfg.D_I, cfg.topk, dsa._dtype_code(g["q_idx"]))
+    ws = dsa.alloc_workspace(ws_bytes or full, dev)
     dsa.dsa_indexer_topk_ranges(g["q_idx"], g["k_idx"], g["w"], torch.tensor(lo, dtype=torch.int32, device=dev),
-                                torch.tensor(hi, dtype=torch.int32, device=dev), cfg.topk, idx, workspace=ws)
+                                torch.tensor(hi, dtype=torch.int32, device=dev), cfg.topk, idx, sc, workspace=ws)
+    if with_scores:
+        return idx.cpu().numpy(), ws, sc.cpu().numpy()
     return idx.cpu().numpy(), ws
 
 
@@ -124,3 +127,25 @@ def test_invalid_range_is_flagged_and_empty():
     pb = oracle_problem(cfg, inp)
     for t in (0, 2, 4, 5, 6, 7):
         check_range_row(pb, idx[t], t, lo[t], hi[t], exact=True)
+
+
+def test_ranges_forced_fallback_is_bit_identical():
+    """Windows of several lengths with a candidate capacity below top-k: every query whose window needs the pilot
+    threshold is rescored by the exact fallback, which scores with the main pass's arithmetic, so indices and
+    scores equal those of the run without a fallback bit for bit."""
+    cfg = dsa_inputs.small_variant(dsa_inputs.CTX128K, N=30000, L=200, topk=512)
+    inp = dsa_inputs.generate(cfg, with_mla=False)
+    lo = [max(0, cfg.q_pos0 + t + 1 - (9000 + 97 * t)) for t in range(cfg.L)]
+    hi = [cfg.q_pos0 + t + 1 for t in range(cfg.L)]
+    idx_a, ws_a, sc_a = run_ranges(cfg, inp, lo, hi, with_scores=True)
+    assert dsa.dsa_workspace_status(ws_a) == 0
+    assert dsa.dsa_workspace_selection_stats(ws_a)["fallback_queries"] == 0
+    full = dsa.dsa_indexer_topk_workspace(cfg.L, cfg.N, cfg.H_I, cfg.D_I, cfg.topk)
+    small = full - cfg.L * (8192 - 256) * 8  # candidate capacity 256 < top-k
+    idx_b, ws_b, sc_b = run_ranges(cfg, inp, lo, hi, ws_bytes=small, with_scores=True)
+    assert dsa.dsa_workspace_status(ws_b) == 0
+    assert dsa.dsa_workspace_selection_stats(ws_b)["fallback_queries"] == cfg.L
+    assert np.array_equal(idx_a, idx_b) and np.array_equal(sc_a, sc_b)
+    pb = oracle_problem(cfg, inp)
+    for t in (0, 99, 199):
+        check_range_row(pb, idx_b[t], t, lo[t], hi[t], exact=False)

@@ -83,3 +83,17 @@ def test_tiny_workload_scales():
     assert _std(inp["w"]) == pytest.approx(0.5, rel=0.1)
     assert _std(inp["kv"][:, :512]) == pytest.approx(0.5, rel=0.03)
     assert _std(inp["kv"][:, 512:]) == pytest.approx(1.0, rel=0.05)
+
+
+def test_correlated_stress_input_is_a_random_walk_over_queries():
+    """The overlap stress input: neighbouring queries' indexer rows and weights differ by 0.05 N(0, 1) steps."""
+    cfg = di.small_variant(di.CORRELATED, N=4096, L=200, H=8)
+    assert cfg.name.startswith("dsa-correlated") and di.CORRELATED not in di.WORKLOADS
+    inp = di.generate(cfg, with_mla=False)
+    q = inp["q_idx"].float()
+    step = q[1:] - q[:-1]
+    assert _std(step) == pytest.approx(di.WALK_STEP, rel=0.1)   # bf16 rounding adds a little
+    assert _std(q[0]) == pytest.approx(1.0, rel=0.15)
+    assert _std(inp["k_idx"]) == pytest.approx(1.0, rel=0.02)
+    w = inp["w"]
+    assert _std(w[1:] - w[:-1]) == pytest.approx(di.WALK_STEP / math.sqrt(cfg.H_I), rel=0.1)

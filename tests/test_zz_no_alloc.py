@@ -1,9 +1,12 @@
 """dsa_indexer_topk_noalloc: the workspace-free indexer top-k for callers that cannot allocate device memory.
 
-Such callers (code running under CUDA graph capture, runtimes that plan every
-byte up front, fully reserved devices) get their scratch from a fixed device
-array inside the library instead of a caller-provided workspace.  This file is
-collected last on purpose; it must pass both alone and after the other tests.
+Such callers (a runtime that plans every byte up front and hands kernels only
+their inputs and outputs, or a device fully reserved by others) get their
+scratch from a fixed device array inside the library instead of a
+caller-provided workspace.  The selection does not depend on the query blocking
+or on which queries go through the exact fallback, so the entry point's output
+must equal the workspace entry point's bit for bit.  This file is collected
+last on purpose; it must pass both alone and after the other tests.
 """
 import numpy as np
 import pytest
@@ -27,36 +30,22 @@ def _selections(cfg):
         idx = torch.full((cfg.L, cfg.topk), -7, dtype=torch.int32, device=dev)
         sc = torch.full((cfg.L, cfg.topk), float("nan"), dtype=torch.float32, device=dev)
         dsa.dsa_indexer_topk_noalloc(q_idx, k_idx, w, cfg.q_pos0, cfg.topk, idx, sc)
-        torch.cuda.synchronize()
+        assert dsa.dsa_indexer_topk_noalloc_status() == 0  # no device-side condition in the fixed scratch
         runs.append((idx.cpu().numpy(), sc.cpu().numpy()))
     return ref_idx.cpu().numpy(), ref_sc.cpu().numpy(), runs
-
-
-def _same_selection(a_idx, a_sc, b_idx, b_sc, rel=1e-6):
-    """Equal sets, except swaps of keys whose scores lie within rel of the k-th score (the tests' tolerance)."""
-    for t in range(a_idx.shape[0]):
-        a, b = a_idx[t][a_idx[t] >= 0], b_idx[t][b_idx[t] >= 0]
-        assert len(a) == len(b)
-        kth = np.min(a_sc[t][a_idx[t] >= 0])
-        if np.array_equal(a, b):
-            np.testing.assert_allclose(b_sc[t][: len(b)], a_sc[t][: len(a)], rtol=1e-5, atol=1e-5 * abs(kth))
-            continue
-        score = dict(zip(a.tolist(), a_sc[t][: len(a)].tolist()))
-        score.update(zip(b.tolist(), b_sc[t][: len(b)].tolist()))
-        for k in np.setxor1d(a, b):
-            assert abs(score[int(k)] - kth) <= rel * abs(kth), f"query {t}: key {k} is not a near-tie swap"
 
 
 @pytest.mark.parametrize("cfg", [
     dsa_inputs.small_variant(dsa_inputs.CTX128K, N=40000, L=300, topk=2048),
     dsa_inputs.small_variant(dsa_inputs.TIES, N=16384, L=130, topk=2048),
+    dsa_inputs.small_variant(dsa_inputs.CTX64K, N=30000, L=200, topk=2048),
     dsa_inputs.CTX128K,
-], ids=["bf16-N40000-L300", "ties-N16384-L130", "bf16-N131072-L1024"])
+], ids=["bf16-N40000-L300", "ties-N16384-L130", "fp8-N30000-L200", "bf16-N131072-L1024"])
 def test_noalloc_matches_workspace_entry_point(cfg):
     ref_idx, ref_sc, runs = _selections(cfg)
     for idx, sc in runs:
-        _same_selection(ref_idx, ref_sc, idx, sc)
-    assert np.array_equal(runs[0][0], runs[1][0])
+        assert np.array_equal(idx, ref_idx)
+        assert np.array_equal(sc, ref_sc)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
