@@ -7,6 +7,10 @@ queries).  Prints one JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
+With --gpus N > 1 and no torch.distributed environment (RANK / WORLD_SIZE
+unset), bench.py starts the N ranks itself under torch.distributed.run on this
+node (127.0.0.1) and passes its exit status on.
+
 Timing: W untimed warm-up steps; then K steps, each preceded by a 512 MiB
 device write that flushes the 126 MB L2, each bracketed by CUDA events on the
 launching stream (the flush is outside the events); a barrier and a device
@@ -173,6 +177,65 @@ def job_throughput(tokens_per_rank: int, world: int, steps: int, max_total_ms: f
     return world * tokens_per_rank * steps / (max_total_ms / 1000.0)
 
 
+def spawn_ranks(gpus: int, argv: list[str]) -> int:
+    """Re-run this script as `gpus` ranks under torch.distributed.run on this node; returns the exit status."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    log(f"[bench] starting {gpus} ranks: {' '.join(cmd)}")
+    return subprocess.call(cmd)
+
+
+def measure_fp8_peak(dev, n: int = 8192, reps: int = 10) -> float | None:
+    """Dense e4m3 tensor throughput on this GPU (TFLOP/s): torch._scaled_mm of two n x n e4m3 matrices with
+    bf16 output, best of `reps` CUDA-event-timed calls (2 n^3 flops each).  None if the call is unavailable."""
+    try:
+        g = torch.Generator(device=dev).manual_seed(7)
+        a = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        run = lambda: torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        for _ in range(3):
+            run()
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            run()
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b
+        return 2.0 * n ** 3 / (best / 1000.0) / 1e12
+    except (RuntimeError, TypeError) as e:
+        log(f"[bench] fp8 peak not measured: {e}")
+        return None
+
+
+def run_dry(args, rank: int, world: int) -> None:
+    """The launch and cross-rank plumbing alone, on CPU ranks (gloo): every rank 'times' a fixed sleep per step,
+    the slowest rank's total is taken, rank 0 prints the JSON line.  Used by the CPU tests of the launcher."""
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("gloo")
+    cfg = dsa_inputs.BY_NAME[args.workload]
+    per_step_s = 0.001 * (1 + rank)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time.sleep(per_step_s)
+    total_ms = max_over_ranks((time.perf_counter() - t0) * 1000.0, world)
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "metric": METRIC, "n_gpus": world, "steps": args.steps,
+                          "ms_per_step": total_ms / args.steps,
+                          "value": job_throughput(cfg.L, world, args.steps, total_ms), "unit": UNIT}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def cpu_oracle_rate(cfg, inp, rows: list[int], threads: int) -> tuple[float, float]:
     """Query tokens/s of the unmodified oracle over `rows` on `threads` host threads; returns (rate, seconds)."""
     import oracle
@@ -305,6 +368,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
 
     step_ms = [starts[k].elapsed_time(ends[k]) for k in range(args.steps)]
     total_ms = sum(step_ms)
+    sel = dsa.dsa_workspace_selection_stats(ws)  # the last timed step's selection totals
     # per-stage times (ms per step, summed over query blocks)
     stage_names = ["pilot", "threshold", "indexer_main", "select", "fallback", "mla"]
     stages = {n: 0.0 for n in stage_names}
@@ -380,10 +444,17 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     launches_per_step = nblocks
     idx_flop_per_launch = fb["indexer_flop"] / launches_per_step
     achieved = idx_flop_per_launch / (main_ms / 1000.0) / 1e12
-    peak = peaks["bf16_tflops"] * (2.0 if cfg.idx_dtype == "e4m3" else 1.0)
+    fp8_peak = measure_fp8_peak(dev) if cfg.idx_dtype == "e4m3" else None
+    if cfg.idx_dtype != "e4m3":
+        peak, peak_source = peaks["bf16_tflops"], f"{peaks['source']} bf16 burst"
+    elif fp8_peak is not None:
+        peak, peak_source = fp8_peak, "measured live: torch._scaled_mm e4m3 8192^3, best of 10"
+    else:
+        peak, peak_source = 2.0 * peaks["bf16_tflops"], f"{peaks['source']} bf16 burst x2 nominal fp8 ratio"
     traffic = indexer_kernel_traffic(cfg)
     # whole-path roofline: max(tensor time at peak, algorithmic bytes at HBM bandwidth)
     t_tensor = (fb["indexer_flop"] / (peak * 1e12)) + fb["mla_flop"] / (peaks["bf16_tflops"] * 1e12)
+    # (the indexer FLOPs at their own dtype's peak, the attention FLOPs at the bf16 peak)
     t_bytes = fb["alg_bytes"] / (peaks["hbm_gbs"] * 1e9)
     path_roof_s = max(t_tensor, t_bytes)
 
@@ -393,9 +464,13 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         n_rows = max(4, min(cfg.L, 16 * threads))  # about 10-15 s of wall time on the 128K workload
         rows = sample_rows(cfg, n_rows)
         rate, secs = cpu_oracle_rate(cfg, inp, rows, threads)
+        rows1 = sample_rows(cfg, 8, salt=77)  # a few seconds on one core
+        rate1, secs1 = cpu_oracle_rate(cfg, inp, rows1, 1)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"{len(rows)} seeded-random query rows of {cfg.name} (full indexer row, exact top-k, "
-                         f"attention), {secs:.1f} s wall on {threads} threads"}
+                         f"attention), {secs:.1f} s wall on {threads} threads",
+               "single_core": {"value": rate1, "unit": UNIT, "cores": 1,
+                               "sample": f"{len(rows1)} seeded-random query rows, {secs1:.1f} s on one thread"}}
 
     pilot_launches = 1 if cfg.q_pos0 + min(cfg.L, 1024) > 8192 else 0
     # Per query block: [pilot], threshold, main pass, select, fallback, attention; a chunk with
@@ -405,7 +480,9 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     gpu_launches = args.steps * nblocks * (5 + pilot_launches + (1 if split else 0))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "ms_per_step_median": statistics.median(step_ms), "ms_per_step_best": min(step_ms),
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg.idx_dtype if cfg.idx_dtype == "bf16" else "fp8-e4m3 indexer / bf16 MLA",
         "data": "synthetic",
         "config": {"workload": cfg.name, "N": cfg.N, "L": cfg.L, "topk": cfg.topk, "H": cfg.H, "H_I": cfg.H_I,
@@ -415,8 +492,11 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "indexer_kernel (main pass)",
-                     "peak_source": f"{peaks['source']} bf16 burst" + (" x2 nominal fp8 ratio" if cfg.idx_dtype == "e4m3" else ""),
+                     "peak_source": peak_source,
                      "path_frac": path_roof_s / (ms_per_step / 1000.0)},
+        "selection": {"candidates_per_query": sel["candidates"] / max(1, sel["queries"]),
+                      "max_candidates": sel["max_candidates"], "fallback_queries": sel["fallback_queries"],
+                      "queries": sel["queries"], "of": "the last timed step"},
         "stages_ms": {k: round(v, 4) for k, v in stages.items()},
         "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -482,6 +562,33 @@ def run_crossover(args) -> None:
         del g, out, ws, wsd, dense_idx
 
 
+def run_overlap(args) -> None:
+    """Neighbouring-query overlap of the selections (measurement only, one JSON line per input): for each pair of
+    consecutive queries t, t + 1, the union ratio |A u B| / (|A| + |B|) of their top-k sets (0.5 = identical sets,
+    1.0 = disjoint).  Packing two queries over their union pays only when this ratio is low."""
+    import numpy as np
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    import deepseek_sparse_attention_relu_b200 as dsa
+    for cfg in (dsa_inputs.CTX64K, dsa_inputs.CTX128K, dsa_inputs.CTX256K, dsa_inputs.CORRELATED):
+        inp = dsa_inputs.generate(cfg, with_mla=False)
+        g = {k: v.to(dev) for k, v in inp.items()}
+        idx = torch.empty(cfg.L, cfg.topk, dtype=torch.int32, device=dev)
+        dsa.dsa_indexer_topk(g["q_idx"], g["k_idx"], g["w"], cfg.q_pos0, cfg.topk, idx)
+        h = idx.cpu().numpy()
+        ratios = np.empty(cfg.L - 1)
+        for t in range(cfg.L - 1):
+            a, b = h[t][h[t] >= 0], h[t + 1][h[t + 1] >= 0]
+            inter = np.intersect1d(a, b, assume_unique=True).size
+            ratios[t] = (a.size + b.size - inter) / (a.size + b.size)
+        print(json.dumps({"overlap": True, "workload": cfg.name, "pairs": int(ratios.size),
+                          "union_ratio_mean": float(ratios.mean()), "union_ratio_min": float(ratios.min()),
+                          "union_ratio_p10": float(np.percentile(ratios, 10)),
+                          "shared_keys_mean": float(cfg.topk * (2 - 2 * ratios.mean())),
+                          "pairs_at_or_below_0.75": int((ratios <= 0.75).sum())}), flush=True)
+        del g, idx
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -492,17 +599,28 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--crossover", action="store_true",
                     help="measure the dense-vs-sparse crossover instead (JSON line per context length)")
+    ap.add_argument("--overlap", action="store_true",
+                    help="measure neighbouring queries' selection overlap instead (JSON line per input)")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="launch and cross-rank plumbing only, on CPU ranks (gloo); no GPU work")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(spawn_ranks(args.gpus, sys.argv[1:]))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         log(f"[bench] note: WORLD_SIZE={world} but --gpus={args.gpus}; using WORLD_SIZE")
-    if args.crossover:
+    if args.dry_run:
+        run_dry(args, rank, world)
+    elif args.crossover:
         if rank == 0:
             run_crossover(args)
+    elif args.overlap:
+        if rank == 0:
+            run_overlap(args)
     elif args.impl == "reference":
         run_reference(args, rank, world)
     else:

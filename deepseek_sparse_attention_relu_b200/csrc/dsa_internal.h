@@ -165,9 +165,6 @@ struct PackArgs {
 cudaError_t launch_pack_plan(const PackArgs &a, cudaStream_t stream);
 
 cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, bool packed, cudaStream_t stream);
-// The unpacked attention on CTA pairs (the 576-wide contraction split over a
-// cluster of two CTAs); no work list.
-cudaError_t launch_sparse_mla_pair(const CUtensorMap &tq, const MlaArgs &a, cudaStream_t stream);
 cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t stream);
 
 }  // namespace dsa

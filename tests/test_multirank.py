@@ -68,3 +68,18 @@ def test_reference_arm_json_line():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "tokens/s"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_bench_starts_its_own_ranks():
+    """`bench.py --gpus 2` without a torch.distributed environment starts two ranks itself (torch.distributed.run
+    on 127.0.0.1); the dry run exercises that launch and the cross-rank max on CPU ranks."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR",
+                                                           "MASTER_PORT")}
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--steps", "5",
+                          "--warmup", "3", "--dry-run"], capture_output=True, text=True, env=env, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(ln) for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1  # rank 0 alone prints
+    line = lines[0]
+    assert line["dry_run"] and line["n_gpus"] == 2 and line["steps"] == 5
+    assert line["ms_per_step"] >= 2.0 * 0.9  # the slower rank (2 ms per step) sets the time
