@@ -351,11 +351,6 @@ dsa_status_t check_mla_args(const MlaProblem &p) {
   return DSA_OK;
 }
 
-bool make_mla_maps(const MlaProblem &p, CUtensorMap *tq) {
-  return make_map_2d(tq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 576, static_cast<uint64_t>(p.L) * p.H, 576 * 2, 64,
-                     64);
-}
-
 // ---- query packing for the attention stage (LiteDSA-style candidate reuse)
 constexpr int kPackMaxEntries = 8192;  // G * topk selection entries per pack (bounds the union)
 constexpr float kMaxUnionRatio = 0.75f; // pack when the union is at most 75% of the members' keys
@@ -419,10 +414,11 @@ size_t attention_scratch_bytes(int L, int QB, int H, int topk) {
   return std::max(b, split_bytes(std::min(L, QB), H, mla_splits(L, H, topk)));
 }
 
-dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, unsigned *status, int t0, int Lq,
-                           cudaStream_t stream, UnionWorkspace uw = UnionWorkspace()) {
+dsa_status_t run_mla_block(const MlaProblem &p, unsigned *status, int t0, int Lq, cudaStream_t stream,
+                           UnionWorkspace uw = UnionWorkspace()) {
   // p.L is the whole chunk's query count (see mla_splits).
   MlaArgs a{};
+  a.q = static_cast<const uint16_t *>(p.q);
   a.topk_idx = p.topk_idx;
   a.kv = p.kv;
   a.kv_ld = p.kv_ld();
@@ -444,7 +440,7 @@ dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, unsigned 
     a.nsplit = ns;
     a.part_o = static_cast<float *>(uw.base);
     a.part_lse = reinterpret_cast<float *>(static_cast<uint8_t *>(uw.base) + align256(rows * 512 * 4));
-    if (!cuda_ok(launch_sparse_mla(tq, a, false, stream))) return DSA_ERR_CUDA;
+    if (!cuda_ok(launch_sparse_mla(a, false, stream))) return DSA_ERR_CUDA;
     return cuda_ok(launch_mla_combine(a, stream)) ? DSA_OK : DSA_ERR_CUDA;
   }
   const int G = pack_group(p.H, p.topk, p.L, p.N);
@@ -481,14 +477,14 @@ dsa_status_t run_mla_block(const MlaProblem &p, const CUtensorMap &tq, unsigned 
     a.ucount = pa.ucount;
     a.list = pa.plist;
     a.list_count = pa.pcount;
-    if (!cuda_ok(launch_sparse_mla(tq, a, true, stream))) return DSA_ERR_CUDA;
+    if (!cuda_ok(launch_sparse_mla(a, true, stream))) return DSA_ERR_CUDA;
     MlaArgs single = a;
     single.G = 1;
     single.list = pa.slist;
     single.list_count = pa.scount;
-    return cuda_ok(launch_sparse_mla(tq, single, false, stream)) ? DSA_OK : DSA_ERR_CUDA;
+    return cuda_ok(launch_sparse_mla(single, false, stream)) ? DSA_OK : DSA_ERR_CUDA;
   }
-  return cuda_ok(launch_sparse_mla(tq, a, false, stream)) ? DSA_OK : DSA_ERR_CUDA;
+  return cuda_ok(launch_sparse_mla(a, false, stream)) ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // namespace
@@ -583,14 +579,12 @@ dsa_status_t dsa_sparse_mla_prefill(const void *q, const void *kv, int64_t ldkv,
   if (st != DSA_OK) return st;
   if (workspace == nullptr || workspace_bytes < kHeaderBytes) return DSA_ERR_WORKSPACE;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  CUtensorMap tq;
-  if (!make_mla_maps(p, &tq)) return DSA_ERR_CUDA;
   unsigned *status = static_cast<unsigned *>(workspace);
   if (!cuda_ok(cudaMemsetAsync(status, 0, kHeaderBytes, stream))) return DSA_ERR_CUDA;
   UnionWorkspace uw;
   uw.base = static_cast<uint8_t *>(workspace) + kHeaderBytes;
   uw.bytes = workspace_bytes - kHeaderBytes;
-  return run_mla_block(p, tq, status, 0, L, stream, uw);
+  return run_mla_block(p, status, 0, L, stream, uw);
 }
 
 size_t dsa_prefill_chunk_workspace(int L, int N, int H_I, int D_I, int H, int topk, int query_block,
@@ -651,8 +645,8 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, int64_t ld
   IdxWorkspace ws;
   if (!carve_idx_ws(workspace, idx_bytes, QB, N, &ws)) return DSA_ERR_WORKSPACE;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  CUtensorMap tq, tk, mq;
-  if (!make_indexer_maps(ip, &tq, &tk) || !make_mla_maps(mp, &mq)) return DSA_ERR_CUDA;
+  CUtensorMap tq, tk;
+  if (!make_indexer_maps(ip, &tq, &tk)) return DSA_ERR_CUDA;
   const int nblocks = (L + QB - 1) / QB;
   if (events != nullptr && n_events < 7 * nblocks) return DSA_ERR_INVALID_ARG;
   if (!cuda_ok(cudaMemsetAsync(ws.status, 0, kHeaderBytes, stream))) return DSA_ERR_CUDA;
@@ -668,7 +662,7 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, int64_t ld
     }
     st = run_indexer_block(bp, tq, tk, ws, t0, Lb, stream, ev);
     if (st != DSA_OK) return st;
-    st = run_mla_block(bm, mq, ws.status, t0, Lb, stream, uw);
+    st = run_mla_block(bm, ws.status, t0, Lb, stream, uw);
     if (st != DSA_OK) return st;
     if (!mark(ev, 6, stream)) return DSA_ERR_CUDA;
   }

@@ -122,6 +122,7 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream);
 
 // Sparse absorbed-MLA attention.
 struct MlaArgs {
+  const uint16_t *q;              // [L, H, 576] bf16 bits: per head 512 latent then 64 rope
   const int32_t *topk_idx;        // [L, topk]
   const void *kv;                 // [N, 576] bf16 joined cache, rows kv_ld elements apart
   long long kv_ld;
@@ -164,7 +165,7 @@ struct PackArgs {
 
 cudaError_t launch_pack_plan(const PackArgs &a, cudaStream_t stream);
 
-cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, bool packed, cudaStream_t stream);
+cudaError_t launch_sparse_mla(const MlaArgs &a, bool packed, cudaStream_t stream);
 cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t stream);
 
 }  // namespace dsa

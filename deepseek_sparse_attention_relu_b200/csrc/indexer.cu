@@ -203,6 +203,9 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
   using C = IdxCfg<DI, HI, FP8>;
   constexpr bool PILOT = MODE == kIdxPilot;
   constexpr bool FB = MODE == kIdxFallback;
+  // No query to rescore (the usual case): leave before any set-up.  The count
+  // was written by the selection kernel, which has completed.
+  if (FB && *reinterpret_cast<volatile int *>(&a.fb_counters[0]) == 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *q_s = smem + C::OFF_Q;

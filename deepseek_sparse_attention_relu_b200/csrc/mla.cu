@@ -11,7 +11,11 @@
 //     out[t,h] = sum_j softmax(z)_j * kv_lat[i_j]          (512 wide)
 // Index -1 marks a skipped entry (llama.cpp PR #25917, discussion).
 //
-// B200 mapping.  One CTA per (query, group of 64 heads).  Per 64-key tile:
+// B200 mapping.  One CTA per (query, group of 64 heads).  Q lives in tensor
+// memory for the whole CTA: the softmax warps copy its 64 x 576 bf16 rows
+// there once, and S = Q K^T reads its A operand from tensor memory, so shared
+// memory holds only gathered keys (three 72 KB stages) and the S MMAs read
+// only the key tile from it.  Per 64-key tile:
 //   * eleven producer warps gather the 64 selected rows with 16-byte cp.async
 //     copies straight into the 128-byte-swizzled UMMA operand layout, two
 //     rows x 256 bytes per warp instruction, with asynchronous per-lane
@@ -21,8 +25,8 @@
 //   * softmax warps read S from TMEM (two lanes per head row, 32 key columns
 //     each), keep a running max (rescaling the output only when the max grows
 //     by more than 2^8) and write P (bf16) in the UMMA layout into the rope
-//     chunk of the tile's own stage (dead once S is done), so P is
-//     double-buffered with the stages at no extra shared memory;
+//     chunk of the tile's own stage (dead once S is done), so P is buffered
+//     with the stages at no extra shared memory;
 //   * O += P V on tcgen05 (M = 64, N = 2 x 256 latent columns, K = 64 keys),
 //     V read in place from the gathered tile as an MN-major operand.
 // The producers also pull the next tile's rows from HBM into L2
@@ -31,11 +35,11 @@
 // mode (chunks with few queries, e.g. decode): CTA z of a query attends its
 // z-th share of the selection and writes a normalised fp32 partial and its
 // log-sum-exp; mla_combine_kernel merges the shares.
-// TMEM: the two 64 x 256 fp32 halves of O sit in the two half-subpartitions
-// (lanes 0-15 and 16-31 of each 32-lane quarter) of columns 0-255, the two S
-// buffers in columns 256-383.  Warp roles: warp 0 MMA issuer / TMEM owner,
-// warps 1-11 gather producers (all of them fill every tile), warps 12-15
-// softmax and output.
+// TMEM (M = 64 operands occupy one 16-lane half of each 32-lane quarter):
+// lanes 0-15 hold Q (columns 0-287, two bf16 per column) and the two S buffers
+// (columns 288-415); lanes 16-31 hold O (columns 0-511).  Warp roles: warp 0
+// MMA issuer / TMEM owner, warps 1-11 gather producers (all of them fill every
+// tile), warps 12-15 Q load, softmax and output.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -51,23 +55,29 @@ constexpr int DIM = 576;         // joined key width
 constexpr int LAT = 512;         // value width
 constexpr int ATOMS = DIM / 64;  // 128-byte column atoms
 constexpr int ATOM_BYTES = 64 * 128;  // 64 rows x 128 B
-constexpr int Q_BYTES = ATOMS * ATOM_BYTES;
 constexpr int KV_BYTES = ATOMS * ATOM_BYTES;
 constexpr int ROPE_OFF = 8 * ATOM_BYTES;  // a stage's rope chunk; holds P once S = Q K^T of its tile is done
-constexpr int STAGES = 2;
+constexpr int STAGES = 3;
 constexpr int N_PROD = 11;                           // gather producer warps
 constexpr int PPW = (BK / 2 + N_PROD - 1) / N_PROD;  // 2-row groups per producer warp
 constexpr int GPW = (BK / 4 + N_PROD - 1) / N_PROD;  // 4-row groups per producer warp
 constexpr int WARP_PROD0 = 1, WARP_SOFT0 = WARP_PROD0 + N_PROD;
 constexpr int THREADS = 32 * (WARP_SOFT0 + 4);
-constexpr int OFF_Q = 0;
-constexpr int OFF_KV = OFF_Q + Q_BYTES;
+constexpr int OFF_KV = 0;
 constexpr int OFF_BAR = OFF_KV + STAGES * KV_BYTES;
-constexpr int NBAR = 1 + 2 * STAGES + 4 + 2 + 1 + STAGES;
+constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 1;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int OFF_VALID = OFF_MISC + 64;            // [STAGES][N_PROD] per-producer-warp key validity words
 constexpr int OFF_MEMB = OFF_VALID + STAGES * N_PROD * 8;  // [STAGES][64] per-query key masks (packed mode)
 constexpr int SMEM_BYTES = OFF_MEMB + STAGES * BK * 8 + 1024;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+// Tensor memory (512 columns; M = 64 operands use one half of each 32-lane
+// quarter): lanes 0-15 hold Q as the A operand of S = Q K^T (576 bf16, two per
+// column: columns 0-287) and the two S buffers (columns 288-351, 352-415);
+// lanes 16-31 hold O (columns 0-511, one per latent dimension).
+constexpr unsigned Q_COL = 0;
+constexpr unsigned S_COL = 288;
+constexpr unsigned O_LANE = 16u << 16;
 constexpr float kRescaleLog2 = 8.0f;
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -80,26 +90,27 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // j*H .. j*H+H-1 of the 64-row tile belong to query j) over the union of their
 // selections; a union key counts for row r only if query r / H chose it.
 template <bool PACKED>
-__global__ void __launch_bounds__(THREADS, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap tmap_q, MlaArgs a) {
+__global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
   pdl_wait_and_release();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *q_s = smem + OFF_Q;
   uint8_t *kv_s = smem + OFF_KV;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-  uint64_t *q_full = bars;
-  uint64_t *kv_full = bars + 1;           // [2]
-  uint64_t *kv_empty = bars + 3;          // [2]
-  uint64_t *s_full = bars + 5;            // [2]
-  uint64_t *s_free = bars + 7;            // [2]
-  uint64_t *p_full = bars + 9;
-  uint64_t *drain = bars + 11;
-  uint64_t *valid_full = bars + 12;       // [2] validity words of the stage's tile published
+  uint64_t *q_full = bars;                     // Q written into tensor memory (one arrival per softmax warp)
+  uint64_t *kv_full = bars + 1;                // [STAGES]
+  uint64_t *kv_empty = bars + 1 + STAGES;      // [STAGES]
+  uint64_t *valid_full = bars + 1 + 2 * STAGES;  // [STAGES] validity words of the stage's tile published
+  uint64_t *s_full = bars + 1 + 3 * STAGES;    // [2]
+  uint64_t *s_free = s_full + 2;               // [2]
+  // [STAGES] P of the stage's tile written.  One barrier per stage: the
+  // softmax may finish two tiles before the MMA warp looks, and with a single
+  // barrier the parity of a phase two ahead would read as "not yet".
+  uint64_t *p_full = s_full + 4;
+  uint64_t *drain = p_full + STAGES;
   unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
-  unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + OFF_VALID);     // [2][N_PROD]
-  unsigned long long *memb_s = reinterpret_cast<unsigned long long *>(smem + OFF_MEMB);       // [2][BK]
+  unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + OFF_VALID);     // [STAGES][N_PROD]
+  unsigned long long *memb_s = reinterpret_cast<unsigned long long *>(smem + OFF_MEMB);       // [STAGES][BK]
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -131,17 +142,17 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int row_limit = PACKED ? nq * a.H : min(HT, a.H - hg * HT);
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(q_full, 4);
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&kv_full[i], N_PROD * 32);  // one asynchronous arrival per producer lane
       mbar_init(&kv_empty[i], 1);
       mbar_init(&valid_full[i], N_PROD);
+      mbar_init(&p_full[i], 4);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
     }
-    mbar_init(p_full, 4);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -150,35 +161,29 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  if (warp == WARP_PROD0 && lane == 0) prefetch_tensormap(&tmap_q);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const unsigned tmem = *tmem_slot;
-  const unsigned o_lo = tmem;                          // lanes 0-15 of each quarter, cols 0-255
-  const unsigned o_hi = tmem + (16u << 16);            // lanes 16-31 of each quarter, cols 0-255
-  const unsigned s_col = tmem + 256;                   // S buffers: cols 256-319, 320-383
+  const unsigned s_col = tmem + S_COL;                 // S buffers (lanes 0-15 of each quarter)
+  const unsigned o_lat0 = tmem + O_LANE;               // O, latent dims 0-255 (lanes 16-31)
+  const unsigned o_lat1 = tmem + O_LANE + 256;         // O, latent dims 256-511
 
   if (warp >= WARP_PROD0 && warp < WARP_SOFT0) {
     // ------------------------------------------------------------ gather producers
-    // All producer warps fill every tile (tile j goes to stage j % 2).  The
-    // latent chunks go in pairs: a warp instruction moves 2 rows x 256 bytes
-    // (lane / 16 picks the row, lane / 8 % 2 the chunk of the pair, lane % 8
-    // the 16-byte piece), which gathers about twice as fast as 4 rows x 128
-    // bytes; the rope chunk goes 4 rows x 128 bytes.  Producer warp pw takes
-    // row pairs and row quads pw + N_PROD i.  Each lane's arrival on the
-    // stage's barrier fires when its copies land, so the producers never
+    // All producer warps fill every tile (tile j goes to stage j % STAGES).
+    // The latent chunks go in pairs: a warp instruction moves 2 rows x 256
+    // bytes (lane / 16 picks the row, lane / 8 % 2 the chunk of the pair, lane
+    // % 8 the 16-byte piece), which gathers about twice as fast as 4 rows x
+    // 128 bytes; the rope chunk goes 4 rows x 128 bytes.  Producer warp pw
+    // takes row pairs and row quads pw + N_PROD i.  Each lane's arrival on
+    // the stage's barrier fires when its copies land, so the producers never
     // block on data and keep many rows in flight.
     const int pw = warp - WARP_PROD0;
     const int u = lane & 7;
     const int sub2 = lane >> 4, seg = (lane >> 3) & 1;  // pair mapping
     const int sub4 = lane >> 3;                         // quad mapping
     bool ok = true;
-    if (pw == 0 && lane == 0) {
-      mbar_arrive_expect_tx(q_full, Q_BYTES);
-      const int row0 = t * a.H + hg * HT;
-      for (int at = 0; at < ATOMS; ++at) tma_load_2d(q_s + at * ATOM_BYTES, &tmap_q, q_full, at * 64, row0);
-    }
     auto key_at = [&](int j, int r) -> int {
       const int pos = j * BK + r;
       return (j < ntiles && pos < nkeys) ? keys[pos] : -1;
@@ -211,7 +216,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int j = 0; j < ntiles; ++j) {
       load_keys(j + 1, kp_n, kq_n);
       cm_n = load_mask(j + 1);
-      const int st = j & 1;
+      const int st = j % STAGES;
       unsigned long long vbits = 0;
 #pragma unroll
       for (int i = 0; i < GPW; ++i) {
@@ -222,7 +227,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       vbits |= __shfl_xor_sync(0xffffffffu, vbits, 8);
       vbits |= __shfl_xor_sync(0xffffffffu, vbits, 16);
-      if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1u, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&kv_empty[st], ((j / STAGES) & 1) ^ 1u, abort_flag)) { ok = false; break; }
       // The stage's previous tile has been consumed (its softmax included).
       if (PACKED && pw == 0 && lane < nq) memb_s[st * BK + lane] = cm;
       __syncwarp();
@@ -251,7 +256,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       cp_async_arrive_noinc(&kv_full[st]);
       // Pull the next tile's rows from HBM into L2 now; its gather starts only
-      // once the other stage is consumed, about half a stage cycle from here.
+      // once its stage is consumed.
 #pragma unroll
       for (int i = 0; i < GPW; ++i) {
         const int v = kq_n[i];
@@ -272,33 +277,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
       *abort_flag = 1;
     }
-    if (pw == 0 && lane == 0 && !mbar_wait(q_full, 0u, nullptr)) atomicOr(a.status, DEV_TIMEOUT);
     __syncwarp();
   } else if (warp == 0) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr unsigned idesc_qk = make_idesc(HT, BK, 1u, 0u, 0u);   // S = Q K^T, both K-major
+    constexpr unsigned idesc_qk = make_idesc(HT, BK, 1u, 0u, 0u);   // S = Q K^T, Q from TMEM, K K-major
     constexpr unsigned idesc_pv = make_idesc(HT, 256, 1u, 0u, 1u);  // O += P V, V MN-major
     bool ok = mbar_wait(q_full, 0u, abort_flag);
-    // Descriptors are built once; an operand offset is added to the start
-    // address field (address >> 4; shared addresses stay below 2^18, so the
-    // 14-bit field never carries).
-    const uint64_t q_desc = smem_desc_sw128(smem_u32(q_s), 16, 1024);
-    const uint64_t p_desc[2] = {smem_desc_sw128(smem_u32(kv_s + ROPE_OFF), 16, 1024),
-                                smem_desc_sw128(smem_u32(kv_s + KV_BYTES + ROPE_OFF), 16, 1024)};
-    const uint64_t k_desc[2] = {smem_desc_sw128(smem_u32(kv_s), 16, 1024),
-                                smem_desc_sw128(smem_u32(kv_s + KV_BYTES), 16, 1024)};
-    const uint64_t v_desc[2] = {smem_desc_sw128(smem_u32(kv_s), ATOM_BYTES, 1024),
-                                smem_desc_sw128(smem_u32(kv_s + KV_BYTES), ATOM_BYTES, 1024)};
+    tc_fence_after();
+    // Descriptors of stage 0; a stage's operands sit KV_BYTES further on,
+    // added to the start-address field (address >> 4; shared addresses stay
+    // below 2^18, so the 14-bit field never carries).
+    const uint64_t k_desc0 = smem_desc_sw128(smem_u32(kv_s), 16, 1024);
+    const uint64_t v_desc0 = smem_desc_sw128(smem_u32(kv_s), ATOM_BYTES, 1024);
+    const uint64_t p_desc0 = smem_desc_sw128(smem_u32(kv_s + ROPE_OFF), 16, 1024);
     auto issue_pv = [&](int jj) {
-      const uint64_t vd = v_desc[jj & 1];
-      const uint64_t pd = p_desc[jj & 1];
+      const int s = jj % STAGES;
+      const uint64_t so = static_cast<uint64_t>((s * KV_BYTES) >> 4);
 #pragma unroll
       for (int ks = 0; ks < BK / 16; ++ks) {
         const unsigned acc = (jj > 0 || ks > 0) ? 1u : 0u;
-        mma_bf16_ss(o_lo, pd + ((ks * 32) >> 4), vd + ((ks * 2048) >> 4), idesc_pv, acc);
-        mma_bf16_ss(o_hi, pd + ((ks * 32) >> 4), vd + ((4 * ATOM_BYTES + ks * 2048) >> 4), idesc_pv, acc);
+        mma_bf16_ss(o_lat0, p_desc0 + so + ((ks * 32) >> 4), v_desc0 + so + ((ks * 2048) >> 4), idesc_pv, acc);
+        mma_bf16_ss(o_lat1, p_desc0 + so + ((ks * 32) >> 4), v_desc0 + so + ((4 * ATOM_BYTES + ks * 2048) >> 4),
+                    idesc_pv, acc);
       }
-      tc_commit(&kv_empty[jj & 1]);
+      tc_commit(&kv_empty[s]);
     };
     // Event-driven issue: O += P V for tile np as soon as its P is written (it
     // frees a gather stage), otherwise S = Q K^T for tile nq once its keys have
@@ -310,9 +312,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     while (ok && np < ntiles) {
       int action = 0;
       if (lane == 0) {
-        if (np < nq && mbar_test_wait(p_full, np & 1u))
+        if (np < nq && mbar_test_wait(&p_full[np % STAGES], (np / STAGES) & 1u))
           action = 1;
-        else if (nq < ntiles && mbar_test_wait(&kv_full[nq & 1], (nq >> 1) & 1u) &&
+        else if (nq < ntiles && mbar_test_wait(&kv_full[nq % STAGES], (nq / STAGES) & 1u) &&
                  mbar_test_wait(&s_free[nq & 1], ((nq >> 1) & 1u) ^ 1u))
           action = 2;
         // the gathered rows were written through the generic proxy
@@ -328,18 +330,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       } else if (action == 2) {
         tc_fence_after();
         if (lane == 0) {
-          const int st = nq & 1;
-          const uint64_t kd = k_desc[st];
-          const unsigned s_tmem = s_col + st * 64;
+          const int st = nq % STAGES;
+          const uint64_t kd = k_desc0 + static_cast<uint64_t>((st * KV_BYTES) >> 4);
+          const unsigned s_tmem = s_col + (nq & 1) * 64;
 #pragma unroll
           for (int at = 0; at < ATOMS; ++at) {
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
               const uint64_t off = static_cast<uint64_t>((at * ATOM_BYTES + ks * 32) >> 4);
-              mma_bf16_ss(s_tmem, q_desc + off, kd + off, idesc_qk, (at | ks) ? 1u : 0u);
+              mma_bf16_ts(s_tmem, tmem + Q_COL + at * 32 + ks * 8, kd + off, idesc_qk, (at | ks) ? 1u : 0u);
             }
           }
-          tc_commit(&s_full[st]);
+          tc_commit(&s_full[nq & 1]);
         }
         __syncwarp();
         ++nq;
@@ -362,19 +364,61 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax + output
+    // ------------------------------------------------------------ Q load, softmax, output
     const int quarter = warp & 3;
     const int r16 = lane & 15;
     const int row = quarter * 16 + r16;  // head within the CTA's group
     const unsigned lane_base = static_cast<unsigned>(quarter * 32) << 16;
+    const int half = lane >> 4;          // which 32 of each 64 columns this thread's 16x32bx2 accesses cover
+    {
+      // Q rows into tensor memory as the A operand of S = Q K^T: row `row`
+      // sits in lane quarter*32 + r16, dims 2c and 2c + 1 in column c.
+      // Thread halves take alternate 64-dim runs of the row (the 16x32bx2
+      // store pairs them); rows past the tile's last valid row are zero.
+      const bool qv = row < row_limit;
+      const uint4 *src = reinterpret_cast<const uint4 *>(a.q) + (out_row0 + row) * (DIM / 8);
+      const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t r[32];
+        const int e0 = 128 * ch + 64 * half;  // first dim of this thread's run
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint4 v = qv ? src[e0 / 8 + k] : z4;
+          r[4 * k] = v.x;
+          r[4 * k + 1] = v.y;
+          r[4 * k + 2] = v.z;
+          r[4 * k + 3] = v.w;
+        }
+        tmem_st_16x32bx2_x32(tmem + lane_base + Q_COL + 64 * ch, r);
+      }
+      {
+        uint32_t r[16];
+        const int e0 = 512 + 32 * half;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint4 v = qv ? src[e0 / 8 + k] : z4;
+          r[4 * k] = v.x;
+          r[4 * k + 1] = v.y;
+          r[4 * k + 2] = v.z;
+          r[4 * k + 3] = v.w;
+        }
+        tmem_st_16x32bx2_x16(tmem + lane_base + Q_COL + 256, r);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_full);
+    }
     float m_used = -INFINITY, l = 0.0f, l_exact = 0.0f;  // l: sum of the bf16 P used; l_exact: fp32 sum for the LSE
     bool ok = true;
-    const int c0 = (lane >> 4) * 32;  // this thread's 32 of the tile's 64 key columns
+    const int c0 = half * 32;  // this thread's 32 of the tile's 64 key columns
     for (int j = 0; j < ntiles; ++j) {
       const int sb = j & 1;
+      const int st = j % STAGES;
       if (!mbar_wait(&s_full[sb], (j >> 1) & 1u, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      if (!mbar_wait(&valid_full[sb], (j >> 1) & 1u, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&valid_full[st], (j / STAGES) & 1u, abort_flag)) { ok = false; break; }
       uint32_t sv[32];
       tmem_ld_16x32bx2_x32(s_col + lane_base + sb * 64, sv);
       tmem_ld_wait();
@@ -385,11 +429,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (PACKED) {
         // keys of this tile that the row's own query chose
         const int qj = row / a.H;
-        vbits = qj < nq ? static_cast<unsigned>(memb_s[(j & 1) * BK + qj] >> c0) : 0u;
+        vbits = qj < nq ? static_cast<unsigned>(memb_s[st * BK + qj] >> c0) : 0u;
       } else {
         unsigned long long vw = 0ull;
 #pragma unroll
-        for (int w = 0; w < N_PROD; ++w) vw |= valid_s[(j & 1) * N_PROD + w];
+        for (int w = 0; w < N_PROD; ++w) vw |= valid_s[st * N_PROD + w];
         vbits = static_cast<unsigned>(vw >> c0);
       }
       float z[32];
@@ -424,29 +468,28 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float alpha = rescale ? fast_exp2(m_old - m_used) : 1.0f;
       l = l * alpha + tsum;
       l_exact = l_exact * alpha + tsum_exact;
-      // Rescale O when the running max moved: lanes 0-15 own the O_lo rows and
-      // lanes 16-31 the O_hi rows of the same heads (same alpha).  O is idle
-      // once O += P V of the previous tile (which frees its stage) is done.
+      // Rescale O when the running max moved: both halves of a row (lanes r16
+      // and r16 + 16) take 32 of every 64 columns of the row's O (same
+      // alpha).  O is idle once O += P V of the previous tile is done.
       if (__any_sync(0xffffffffu, rescale)) {
-        if (!mbar_wait(&kv_empty[(j - 1) & 1], ((j - 1) >> 1) & 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&kv_empty[(j - 1) % STAGES], ((j - 1) / STAGES) & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const unsigned obase = o_lo + lane_base;  // one 32x32b access: O_lo rows then O_hi rows
 #pragma unroll 1
         for (int ch = 0; ch < 8; ++ch) {
           uint32_t ov[32];
-          tmem_ld_32x32b_x32(obase + ch * 32, ov);
+          tmem_ld_16x32bx2_x32(o_lat0 + lane_base + ch * 64, ov);
           tmem_ld_wait();
           if (rescale) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
           }
-          tmem_st_32x32b_x32(obase + ch * 32, ov);
+          tmem_st_16x32bx2_x32(o_lat0 + lane_base + ch * 64, ov);
         }
         tmem_st_wait();
       }
       {
         // P of tile j goes into the rope chunk of its own stage (dead after S = Q K^T)
-        uint8_t *prow = kv_s + (j & 1) * KV_BYTES + ROPE_OFF + row * 128;
+        uint8_t *prow = kv_s + st * KV_BYTES + ROPE_OFF + row * 128;
         const int cbase = c0 >> 3;  // first 16-byte chunk of this thread's 32 columns
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -457,9 +500,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[st]);
     }
-    if (ok) ok = mbar_wait(&kv_empty[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1u, abort_flag);
+    if (ok) ok = mbar_wait(&kv_empty[(ntiles - 1) % STAGES], ((ntiles - 1) / STAGES) & 1u, abort_flag);
     if (!ok) {
       if (lane == 0) atomicOr(a.status, DEV_TIMEOUT);
       *abort_flag = 1;
@@ -467,18 +510,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const float inv = l > 0.0f ? 1.0f / l : 0.0f;  // both halves of a row hold the row's l
       const bool has_row = row < row_limit;
-      const int dim0 = lane < 16 ? 0 : 256;
-      uint16_t *orow = a.out + (out_row0 + row) * LAT + dim0;
+      uint16_t *orow = a.out + (out_row0 + row) * LAT;
       // split-key mode: this share's normalised fp32 output row
       const long long prow_idx = (static_cast<long long>(t - a.t0) * a.H + hg * HT + row) * a.nsplit + split;
-      float *porow = split_mode ? a.part_o + prow_idx * LAT + dim0 : nullptr;
+      float *porow = split_mode ? a.part_o + prow_idx * LAT : nullptr;
 #pragma unroll 1
       for (int ch = 0; ch < 8; ++ch) {
         uint32_t ov[32];
-        tmem_ld_32x32b_x32(o_lo + lane_base + ch * 32, ov);
+        tmem_ld_16x32bx2_x32(o_lat0 + lane_base + ch * 64, ov);
         tmem_ld_wait();
+        const int d0 = 64 * ch + c0;  // this thread's 32 latent dims
         if (has_row && split_mode) {
-          float4 *dst = reinterpret_cast<float4 *>(porow + ch * 32);
+          float4 *dst = reinterpret_cast<float4 *>(porow + d0);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
@@ -491,7 +534,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 __floats2bfloat162_rn(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
             pkd[e] = *reinterpret_cast<const uint32_t *>(&b);
           }
-          uint4 *dst = reinterpret_cast<uint4 *>(orow + ch * 32);
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + d0);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
         }
@@ -582,13 +625,13 @@ cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t stream) {
   return launch_kernel(mla::mla_combine_kernel, dim3(blocks), dim3(256), 0, stream, a);
 }
 
-cudaError_t launch_sparse_mla(const CUtensorMap &tq, const MlaArgs &a, bool packed, cudaStream_t stream) {
+cudaError_t launch_sparse_mla(const MlaArgs &a, bool packed, cudaStream_t stream) {
   auto kern = packed ? mla::sparse_mla_kernel<true> : mla::sparse_mla_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(packed ? (a.Lq + a.G - 1) / a.G : a.Lq, packed ? 1 : (a.H + mla::HT - 1) / mla::HT,
             packed ? 1 : max(1, a.nsplit));
-  return launch_kernel(kern, grid, dim3(mla::THREADS), mla::SMEM_BYTES, stream, tq, a);
+  return launch_kernel(kern, grid, dim3(mla::THREADS), mla::SMEM_BYTES, stream, a);
 }
 
 }  // namespace dsa

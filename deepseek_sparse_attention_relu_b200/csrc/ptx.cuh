@@ -175,6 +175,19 @@ __device__ __forceinline__ void mma_fp8_ss(unsigned d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T: A read from tensor memory (K-major, two
+// 16-bit elements per 32-bit column; for M = 64 its rows sit in lanes 0-15 of
+// each 32-lane quarter, offset by the address's lane field).
+__device__ __forceinline__ void mma_bf16_ts(unsigned d_tmem, unsigned a_tmem, uint64_t b_desc, unsigned idesc,
+                                            unsigned accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Instruction descriptor for dense kind::f16 / kind::f8f6f4 with fp32 accumulate.
 // fmt: bf16 = 1 (kind::f16), e4m3 = 0 (kind::f8f6f4).  a_mn / b_mn: operand is
 // MN-major (1) or K-major (0).
@@ -234,6 +247,27 @@ __device__ __forceinline__ void tmem_ld_16x32bx2_x32(unsigned taddr, uint32_t (&
         "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
+}
+// Stores matching tmem_ld_16x32bx2_x32 (threads 0-15: lanes base+0..15,
+// columns [col, col + 32); threads 16-31: the same lanes, [col + 32, col + 64)).
+__device__ __forceinline__ void tmem_st_16x32bx2_x32(unsigned taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 32, {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+// Half-width version: threads 0-15 columns [col, col + 16), threads 16-31 [col + 16, col + 32).
+__device__ __forceinline__ void tmem_st_16x32bx2_x16(unsigned taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 16, {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
 }
 // 16 lanes x 256 bit, four repeats along the columns (32 columns in all).  For
 // repeat j, thread t gets r[4j], r[4j+1] = lane base + t/4, columns
