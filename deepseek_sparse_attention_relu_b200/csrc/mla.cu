@@ -50,35 +50,46 @@ namespace dsa {
 namespace mla {
 
 constexpr int HT = 64;           // heads per CTA (UMMA M)
-constexpr int BK = 64;           // keys per tile
 constexpr int DIM = 576;         // joined key width
 constexpr int LAT = 512;         // value width
 constexpr int ATOMS = DIM / 64;  // 128-byte column atoms
-constexpr int ATOM_BYTES = 64 * 128;  // 64 rows x 128 B
-constexpr int KV_BYTES = ATOMS * ATOM_BYTES;
-constexpr int ROPE_OFF = 8 * ATOM_BYTES;  // a stage's rope chunk; holds P once S = Q K^T of its tile is done
-constexpr int STAGES = 3;
-constexpr int N_PROD = 11;                           // gather producer warps
-constexpr int PPW = (BK / 2 + N_PROD - 1) / N_PROD;  // 2-row groups per producer warp
-constexpr int GPW = (BK / 4 + N_PROD - 1) / N_PROD;  // 4-row groups per producer warp
+constexpr int N_PROD = 11;       // gather producer warps
 constexpr int WARP_PROD0 = 1, WARP_SOFT0 = WARP_PROD0 + N_PROD;
 constexpr int THREADS = 32 * (WARP_SOFT0 + 4);
-constexpr int OFF_KV = 0;
-constexpr int OFF_BAR = OFF_KV + STAGES * KV_BYTES;
-constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 1;
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int OFF_VALID = OFF_MISC + 64;            // [STAGES][N_PROD] per-producer-warp key validity words
-constexpr int OFF_MEMB = OFF_VALID + STAGES * N_PROD * 8;  // [STAGES][64] per-query key masks (packed mode)
-constexpr int SMEM_BYTES = OFF_MEMB + STAGES * BK * 8 + 1024;
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 // Tensor memory (512 columns; M = 64 operands use one half of each 32-lane
 // quarter): lanes 0-15 hold Q as the A operand of S = Q K^T (576 bf16, two per
-// column: columns 0-287) and the two S buffers (columns 288-351, 352-415);
-// lanes 16-31 hold O (columns 0-511, one per latent dimension).
+// column: columns 0-287) and the two S buffers (from column 288); lanes 16-31
+// hold O (columns 0-511, one per latent dimension).
 constexpr unsigned Q_COL = 0;
 constexpr unsigned S_COL = 288;
 constexpr unsigned O_LANE = 16u << 16;
 constexpr float kRescaleLog2 = 8.0f;
+
+// Per-variant tiling.  Unpacked: 96-key tiles in two stages (an S MMA of
+// N = 96 costs about what one of N = 64 does, so S = Q K^T takes a third fewer
+// MMA instructions per key).  Packed (H <= 32): 64-key tiles in three stages,
+// matching the pack plan's 64-key union tiles and membership masks.
+template <bool PACKED>
+struct MlaCfg {
+  static constexpr int BK = PACKED ? 64 : 96;          // keys per tile (N of S = Q K^T)
+  static constexpr int STAGES = PACKED ? 3 : 2;
+  static constexpr int ATOM_BYTES = BK * 128;          // BK rows x 128 B
+  static constexpr int KV_BYTES = ATOMS * ATOM_BYTES;
+  static constexpr int ROPE_OFF = 8 * ATOM_BYTES;      // a stage's rope chunk; holds P once S of its tile is done
+  static constexpr int NC = BK / 2;                    // key columns per softmax thread (two threads per row)
+  static constexpr int PPW = (BK / 2 + N_PROD - 1) / N_PROD;  // 2-row groups per producer warp
+  static constexpr int GPW = (BK / 4 + N_PROD - 1) / N_PROD;  // 4-row groups per producer warp
+  static constexpr int OFF_KV = 0;
+  static constexpr int OFF_BAR = OFF_KV + STAGES * KV_BYTES;
+  static constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_VALID = OFF_MISC + 64;      // [STAGES][N_PROD][2] key validity words (128 keys max)
+  static constexpr int OFF_MEMB = OFF_VALID + STAGES * N_PROD * 16;  // [STAGES][64] per-query key masks (packed)
+  static constexpr int SMEM_BYTES = OFF_MEMB + STAGES * 64 * 8 + 1024;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(S_COL + 2 * BK <= 512, "tensor memory budget");
+  static_assert(BK % 32 == 0 && BK <= 128, "tile width");
+};
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -92,10 +103,13 @@ __device__ __forceinline__ float fast_exp2(float x) {
 template <bool PACKED>
 __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
   pdl_wait_and_release();
+  using C = MlaCfg<PACKED>;
+  constexpr int BK = C::BK, STAGES = C::STAGES, ATOM_BYTES = C::ATOM_BYTES, KV_BYTES = C::KV_BYTES;
+  constexpr int ROPE_OFF = C::ROPE_OFF, NC = C::NC, PPW = C::PPW, GPW = C::GPW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *kv_s = smem + OFF_KV;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  uint8_t *kv_s = smem + C::OFF_KV;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
   uint64_t *q_full = bars;                     // Q written into tensor memory (one arrival per softmax warp)
   uint64_t *kv_full = bars + 1;                // [STAGES]
   uint64_t *kv_empty = bars + 1 + STAGES;      // [STAGES]
@@ -107,10 +121,10 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
   // barrier the parity of a phase two ahead would read as "not yet".
   uint64_t *p_full = s_full + 4;
   uint64_t *drain = p_full + STAGES;
-  unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + OFF_MISC);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
-  unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + OFF_VALID);     // [STAGES][N_PROD]
-  unsigned long long *memb_s = reinterpret_cast<unsigned long long *>(smem + OFF_MEMB);       // [STAGES][BK]
+  unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + C::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+  unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + C::OFF_VALID);  // [STAGES][N_PROD][2]
+  unsigned long long *memb_s = reinterpret_cast<unsigned long long *>(smem + C::OFF_MEMB);    // [STAGES][64]
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -217,22 +231,28 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
       load_keys(j + 1, kp_n, kq_n);
       cm_n = load_mask(j + 1);
       const int st = j % STAGES;
-      unsigned long long vbits = 0;
+      unsigned long long vlo = 0, vhi = 0;  // validity of tile rows 0-63, 64-127
 #pragma unroll
       for (int i = 0; i < GPW; ++i) {
         const int v = kq[i];
         if (u == 0 && (v >= a.N || v < -1)) atomicOr(a.status, DEV_BAD_INDEX);
         const int grp = pw + N_PROD * i;
-        if (grp < BK / 4 && v >= 0 && v < a.N) vbits |= 1ull << (4 * grp + sub4);
+        if (grp < BK / 4 && v >= 0 && v < a.N) {
+          const int bit = 4 * grp + sub4;
+          if (bit < 64) vlo |= 1ull << bit; else vhi |= 1ull << (bit - 64);
+        }
       }
-      vbits |= __shfl_xor_sync(0xffffffffu, vbits, 8);
-      vbits |= __shfl_xor_sync(0xffffffffu, vbits, 16);
+      vlo |= __shfl_xor_sync(0xffffffffu, vlo, 8);
+      vlo |= __shfl_xor_sync(0xffffffffu, vlo, 16);
+      vhi |= __shfl_xor_sync(0xffffffffu, vhi, 8);
+      vhi |= __shfl_xor_sync(0xffffffffu, vhi, 16);
       if (!mbar_wait(&kv_empty[st], ((j / STAGES) & 1) ^ 1u, abort_flag)) { ok = false; break; }
       // The stage's previous tile has been consumed (its softmax included).
-      if (PACKED && pw == 0 && lane < nq) memb_s[st * BK + lane] = cm;
+      if (PACKED && pw == 0 && lane < nq) memb_s[st * 64 + lane] = cm;
       __syncwarp();
       if (lane == 0) {
-        valid_s[st * N_PROD + pw] = vbits;
+        valid_s[(st * N_PROD + pw) * 2] = vlo;
+        valid_s[(st * N_PROD + pw) * 2 + 1] = vhi;
         mbar_arrive(&valid_full[st]);
       }
       const unsigned stage_base = smem_u32(kv_s + st * KV_BYTES);
@@ -289,16 +309,22 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
     // below 2^18, so the 14-bit field never carries).
     const uint64_t k_desc0 = smem_desc_sw128(smem_u32(kv_s), 16, 1024);
     const uint64_t v_desc0 = smem_desc_sw128(smem_u32(kv_s), ATOM_BYTES, 1024);
-    const uint64_t p_desc0 = smem_desc_sw128(smem_u32(kv_s + ROPE_OFF), 16, 1024);
+    // P (A of O += P V): 128-byte-swizzled rows for 64-key tiles; for 96-key
+    // tiles the no-swizzle core-matrix layout, which fits 64 x 96 bf16 in the
+    // 12 KB rope chunk (core matrices 128 B apart along K, 8-row groups
+    // BK / 8 * 128 B apart).
+    const uint64_t p_desc0 = BK == 64 ? smem_desc_sw128(smem_u32(kv_s + ROPE_OFF), 16, 1024)
+                                      : smem_desc_noswz(smem_u32(kv_s + ROPE_OFF), 128, BK / 8 * 128);
+    constexpr int P_KSTEP = BK == 64 ? 32 : 256;  // bytes between the P operands of consecutive 16-key steps
     auto issue_pv = [&](int jj) {
       const int s = jj % STAGES;
       const uint64_t so = static_cast<uint64_t>((s * KV_BYTES) >> 4);
 #pragma unroll
       for (int ks = 0; ks < BK / 16; ++ks) {
         const unsigned acc = (jj > 0 || ks > 0) ? 1u : 0u;
-        mma_bf16_ss(o_lat0, p_desc0 + so + ((ks * 32) >> 4), v_desc0 + so + ((ks * 2048) >> 4), idesc_pv, acc);
-        mma_bf16_ss(o_lat1, p_desc0 + so + ((ks * 32) >> 4), v_desc0 + so + ((4 * ATOM_BYTES + ks * 2048) >> 4),
-                    idesc_pv, acc);
+        mma_bf16_ss(o_lat0, p_desc0 + so + ((ks * P_KSTEP) >> 4), v_desc0 + so + ((ks * 2048) >> 4), idesc_pv, acc);
+        mma_bf16_ss(o_lat1, p_desc0 + so + ((ks * P_KSTEP) >> 4),
+                    v_desc0 + so + ((4 * ATOM_BYTES + ks * 2048) >> 4), idesc_pv, acc);
       }
       tc_commit(&kv_empty[s]);
     };
@@ -332,7 +358,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
         if (lane == 0) {
           const int st = nq % STAGES;
           const uint64_t kd = k_desc0 + static_cast<uint64_t>((st * KV_BYTES) >> 4);
-          const unsigned s_tmem = s_col + (nq & 1) * 64;
+          const unsigned s_tmem = s_col + (nq & 1) * BK;
 #pragma unroll
           for (int at = 0; at < ATOMS; ++at) {
 #pragma unroll
@@ -412,35 +438,42 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
     }
     float m_used = -INFINITY, l = 0.0f, l_exact = 0.0f;  // l: sum of the bf16 P used; l_exact: fp32 sum for the LSE
     bool ok = true;
-    const int c0 = half * 32;  // this thread's 32 of the tile's 64 key columns
+    // This thread's NC of the tile's BK key columns: [32 half, 32 half + 32)
+    // and, for 96-key tiles, also [64 + 16 half, 64 + 16 half + 16) (TMEM
+    // half-split loads whose second half sits one load width further on).
+    const int c0 = half * 32;
     for (int j = 0; j < ntiles; ++j) {
       const int sb = j & 1;
       const int st = j % STAGES;
       if (!mbar_wait(&s_full[sb], (j >> 1) & 1u, abort_flag)) { ok = false; break; }
       tc_fence_after();
       if (!mbar_wait(&valid_full[st], (j / STAGES) & 1u, abort_flag)) { ok = false; break; }
-      uint32_t sv[32];
-      tmem_ld_16x32bx2_x32(s_col + lane_base + sb * 64, sv);
+      uint32_t sv[NC];
+      tmem_ld_16x32bx2_x32_split<32>(s_col + lane_base + sb * BK, sv);
+      if constexpr (NC == 48) tmem_ld_16x32bx2_x16_split<16>(s_col + lane_base + sb * BK + 64, sv + 32);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[sb]);
-      unsigned vbits;
+      unsigned long long vbits;  // bit c: this thread's c-th key column holds a valid key
       if (PACKED) {
         // keys of this tile that the row's own query chose
         const int qj = row / a.H;
-        vbits = qj < nq ? static_cast<unsigned>(memb_s[st * BK + qj] >> c0) : 0u;
+        vbits = qj < nq ? (memb_s[st * 64 + qj] >> c0) : 0ull;
       } else {
-        unsigned long long vw = 0ull;
+        unsigned long long lo = 0ull, hi = 0ull;
 #pragma unroll
-        for (int w = 0; w < N_PROD; ++w) vw |= valid_s[st * N_PROD + w];
-        vbits = static_cast<unsigned>(vw >> c0);
+        for (int w = 0; w < N_PROD; ++w) {
+          lo |= valid_s[(st * N_PROD + w) * 2];
+          hi |= valid_s[(st * N_PROD + w) * 2 + 1];
+        }
+        vbits = ((lo >> c0) & 0xFFFFFFFFull) | (((hi >> (16 * half)) & 0xFFFFull) << 32);
       }
-      float z[32];
+      float z[NC];
       float tmax = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        z[c] = ((vbits >> c) & 1u) ? __uint_as_float(sv[c]) * a.scale_log2 : -INFINITY;
+      for (int c = 0; c < NC; ++c) {
+        z[c] = ((vbits >> c) & 1ull) ? __uint_as_float(sv[c]) * a.scale_log2 : -INFINITY;
         tmax = fmaxf(tmax, z[c]);
       }
       tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));  // whole row (both halves)
@@ -451,10 +484,10 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
         m_used = tmax;
       }
       // P in bf16, rounded once; the normaliser sums the rounded values.
-      uint32_t pk[16];
+      uint32_t pk[NC / 2];
       float tsum = 0.0f, tsum_exact = 0.0f;
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
+      for (int c = 0; c < NC; c += 2) {
         const float p0 = (m_used == -INFINITY) ? 0.0f : fast_exp2(z[c] - m_used);
         const float p1 = (m_used == -INFINITY) ? 0.0f : fast_exp2(z[c + 1] - m_used);
         const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
@@ -489,12 +522,15 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
       }
       {
         // P of tile j goes into the rope chunk of its own stage (dead after S = Q K^T)
-        uint8_t *prow = kv_s + st * KV_BYTES + ROPE_OFF + row * 128;
-        const int cbase = c0 >> 3;  // first 16-byte chunk of this thread's 32 columns
+        uint8_t *pbase = kv_s + st * KV_BYTES + ROPE_OFF;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < NC / 8; ++ch) {
           const uint4 v = make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-          *reinterpret_cast<uint4 *>(prow + (((cbase + ch) ^ (row & 7)) << 4)) = v;
+          const int k = ch < 4 ? 4 * half + ch : 8 + 2 * half + (ch - 4);  // 8-key chunk of the tile
+          if constexpr (BK == 64)  // 128-byte-swizzled row
+            *reinterpret_cast<uint4 *>(pbase + row * 128 + ((k ^ (row & 7)) << 4)) = v;
+          else  // core matrix (row / 8, k), row row % 8 within it
+            *reinterpret_cast<uint4 *>(pbase + (row >> 3) * (BK / 8 * 128) + k * 128 + (row & 7) * 16) = v;
         }
       }
       fence_proxy_async_smem();
@@ -627,11 +663,12 @@ cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t stream) {
 
 cudaError_t launch_sparse_mla(const MlaArgs &a, bool packed, cudaStream_t stream) {
   auto kern = packed ? mla::sparse_mla_kernel<true> : mla::sparse_mla_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES);
+  const int smem = packed ? mla::MlaCfg<true>::SMEM_BYTES : mla::MlaCfg<false>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(packed ? (a.Lq + a.G - 1) / a.G : a.Lq, packed ? 1 : (a.H + mla::HT - 1) / mla::HT,
             packed ? 1 : max(1, a.nsplit));
-  return launch_kernel(kern, grid, dim3(mla::THREADS), mla::SMEM_BYTES, stream, a);
+  return launch_kernel(kern, grid, dim3(mla::THREADS), smem, stream, a);
 }
 
 }  // namespace dsa

@@ -248,6 +248,41 @@ __device__ __forceinline__ void tmem_ld_16x32bx2_x32(unsigned taddr, uint32_t (&
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+// 16-lane loads with the second half at a chosen column offset SPLIT: threads
+// 0-15 get lanes base+0..15, columns [col, col + n); threads 16-31 the same
+// lanes, columns [col + SPLIT, col + SPLIT + n).  n = 32 (x32) or 16 (x16).
+template <int SPLIT>
+__device__ __forceinline__ void tmem_ld_16x32bx2_x32_split(unsigned taddr, uint32_t *r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32], %33;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr), "n"(SPLIT));
+}
+template <int SPLIT>
+__device__ __forceinline__ void tmem_ld_16x32bx2_x16_split(unsigned taddr, uint32_t *r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16], %17;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr), "n"(SPLIT));
+}
+
+// Shared-memory matrix descriptor without swizzling (K-major: 8-row x 16-byte
+// core matrices, lbo bytes apart along K, sbo bytes apart along M/N).
+__device__ __forceinline__ uint64_t smem_desc_noswz(unsigned saddr, unsigned lbo, unsigned sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;  // version
+  return d;         // layout type 0: no swizzle
+}
+
 // Stores matching tmem_ld_16x32bx2_x32 (threads 0-15: lanes base+0..15,
 // columns [col, col + 32); threads 16-31: the same lanes, [col + 32, col + 64)).
 __device__ __forceinline__ void tmem_st_16x32bx2_x32(unsigned taddr, const uint32_t (&r)[32]) {
