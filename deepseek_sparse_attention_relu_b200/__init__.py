@@ -296,7 +296,8 @@ def dsa_prefill_chunk_profiled(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torc
                                query_block: int = 0, workspace: torch.Tensor | None = None, stream=None) -> None:
     """dsa_prefill_chunk recording 7 CUDA events per query block between its stages (see include/dsa.h).
 
-    events: torch.cuda.Event objects that have been recorded at least once (so their handles exist)."""
+    events: torch.cuda.Event objects that have been recorded at least once (so their handles exist), or None
+    for a boundary that should not be marked."""
     L, H_I, D_I = q_idx.shape
     N = k_idx.shape[0]
     H = q.shape[1]
@@ -304,7 +305,7 @@ def dsa_prefill_chunk_profiled(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torc
     if workspace is None:
         workspace = alloc_workspace(dsa_prefill_chunk_workspace(L, N, H_I, D_I, H, topk, query_block, dt,
                                                                 topk_idx is not None), q.device)
-    handles = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    handles = (ctypes.c_void_p * len(events))(*[None if e is None else e.cuda_event for e in events])
     _check(lib().dsa_prefill_chunk_profiled(
         _dev(q_idx, "q_idx"), *_rows(k_idx, "k_idx"), _dev(w, "w", (torch.float32,)), dt,
         _dev(q, "q", (torch.bfloat16,)), *_rows(kv, "kv", (torch.bfloat16,)), L, N, H_I, D_I, H, q_pos0, topk,

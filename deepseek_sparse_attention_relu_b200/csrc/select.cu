@@ -31,12 +31,13 @@
 namespace dsa {
 
 constexpr int kSelThreads = 512;
-constexpr int kMaxTopk = 4096;
 
 // ------------------------------------------------------------------ threshold
 constexpr int kMaxSamples = 4096;
 
-__global__ void __launch_bounds__(256) threshold_kernel(SelectArgs a) {
+// 1,024 queries per block and seven CTAs per SM (register and shared-memory
+// budgets sized for it) make the launch a single wave on 148 SMs.
+__global__ void __launch_bounds__(256, 7) threshold_kernel(SelectArgs a) {
   pdl_wait_and_release();
   __shared__ unsigned hist[256];
   __shared__ unsigned misc[4];
@@ -99,14 +100,27 @@ __device__ void block_bitonic_sort(unsigned long long *v, int n) {
 }
 
 // ------------------------------------------------------------------ select
-constexpr int kSmemCand = 8192;        // candidates staged in shared memory (larger lists stay in L2)
-constexpr int kBitmapKeys = 262144;    // ascending output through a shared bitmap up to this many keys
+// Shared memory of the selection kernel, sized per launch so that several of
+// its CTAs share an SM: up to kSmemCand candidates are staged (a longer list is
+// read from L2), then a region that holds either the bitmap over the visible
+// keys (ascending output) or the sort buffer of the selected pairs.
+constexpr int kSmemCand = 6144;
+constexpr int kBitmapMaxKeys = 262144;  // the bitmap path covers caches up to this many keys
+
+int select_stage_cap(const SelectArgs &a) { return min(a.cap, kSmemCand); }
+int select_region_bytes(const SelectArgs &a) {
+  int npow = 1;
+  while (npow < a.topk) npow <<= 1;
+  const int bitmap = a.N <= kBitmapMaxKeys ? (a.N + 31) / 32 * 4 : 0;
+  return max(bitmap, npow * 8);
+}
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   pdl_wait_and_release();
   extern __shared__ __align__(16) unsigned char sel_smem[];
   unsigned long long *cs = reinterpret_cast<unsigned long long *>(sel_smem);         // staged candidates
-  unsigned char *region = sel_smem + static_cast<size_t>(min(a.cap, kSmemCand)) * 8;  // bitmap or sort buffer
+  const int stage_cap = min(a.cap, kSmemCand);
+  unsigned char *region = sel_smem + static_cast<size_t>(stage_cap) * 8;  // bitmap or sort buffer
   __shared__ unsigned hist[256];
   __shared__ unsigned misc[4];
   __shared__ int warp_tot[kSelThreads / 32];
@@ -132,7 +146,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     return;
   }
   const unsigned long long *cand = a.cand + static_cast<long long>(tl) * a.cap;
-  const bool staged = count <= kSmemCand;
+  const bool staged = count <= stage_cap;
   if (staged) {
     for (int i = threadIdx.x; i < count; i += blockDim.x) cs[i] = cand[i];
     __syncthreads();
@@ -143,7 +157,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   int32_t *out = a.topk_idx + static_cast<long long>(t) * a.topk;
   float *osc = a.topk_score ? a.topk_score + static_cast<long long>(t) * a.topk : nullptr;
 
-  if (osc == nullptr && nvis <= kBitmapKeys) {
+  // (the region holds a bitmap over [lo, lo + nvis) whenever N <= kBitmapMaxKeys, since nvis <= N)
+  if (osc == nullptr && a.N <= kBitmapMaxKeys) {
     // Winners -> bitmap over key indices -> ordered compaction (ascending keys).
     unsigned *bitmap = reinterpret_cast<unsigned *>(region);
     const int nwords = (nvis + 31) >> 5;
@@ -386,8 +401,7 @@ cudaError_t launch_threshold(const SelectArgs &a, cudaStream_t stream) {
 }
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream) {
-  // staged candidates + max(bitmap of kBitmapKeys bits, sort buffer of kMaxTopk pairs)
-  const int smem = min(a.cap, kSmemCand) * 8 + max(kBitmapKeys / 8, kMaxTopk * 8);
+  const int smem = select_stage_cap(a) * 8 + select_region_bytes(a);
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   return launch_kernel(select_kernel, dim3(a.Lb), dim3(kSelThreads), smem, stream, a);

@@ -260,7 +260,9 @@ dsa_status_t dsa_prefill_chunk_ranges(const void *q_idx, const void *k_idx, int6
  * n_events >= 7 * ceil(L / query_block) cudaEvent_t handles; for query block b,
  * events[7b + 0..6] are recorded before the pilot pass, after the pilot pass,
  * after the threshold kernel, after the main indexer pass, after the
- * selection, after the exact fallback and after the attention kernel.
+ * selection, after the exact fallback and after the attention kernel.  A NULL
+ * handle leaves that boundary unmarked (an event between two kernels keeps the
+ * second from launching before the first completes).
  */
 dsa_status_t dsa_prefill_chunk_profiled(const void *q_idx, const void *k_idx, int64_t ldk, const float *w,
                                         dsa_dtype_t dtype, const void *q, const void *kv, int64_t ldkv, int L, int N,
