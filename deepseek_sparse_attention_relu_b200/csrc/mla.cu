@@ -14,20 +14,21 @@
 // B200 mapping.  One CTA per (query, group of 64 heads).  Q lives in tensor
 // memory for the whole CTA: the softmax warps copy its 64 x 576 bf16 rows
 // there once, and S = Q K^T reads its A operand from tensor memory, so shared
-// memory holds only gathered keys (three 72 KB stages) and the S MMAs read
-// only the key tile from it.  Per 64-key tile:
-//   * eleven producer warps gather the 64 selected rows with 16-byte cp.async
-//     copies straight into the 128-byte-swizzled UMMA operand layout, two
-//     rows x 256 bytes per warp instruction, with asynchronous per-lane
-//     arrivals; a tensor-map gather (tile::gather4) was measured to issue too
-//     slowly for 1,152-byte rows;
-//   * S = Q K^T on tcgen05 (M = 64 heads, N = 64 keys, K = 576), fp32 in TMEM;
-//   * softmax warps read S from TMEM (two lanes per head row, 32 key columns
+// memory holds only gathered keys (two 108 KB stages of 96-key tiles; the
+// packed variant uses three 72 KB stages of 64 keys) and the S MMAs read only
+// the key tile from it.  Per tile:
+//   * eleven producer warps gather the tile's selected rows with 16-byte
+//     cp.async copies straight into the 128-byte-swizzled UMMA operand
+//     layout, two rows x 256 bytes per warp instruction, with asynchronous
+//     per-lane arrivals; a tensor-map gather (tile::gather4) was measured to
+//     issue too slowly for 1,152-byte rows;
+//   * S = Q K^T on tcgen05 (M = 64 heads, N = 96 keys, K = 576), fp32 in TMEM;
+//   * softmax warps read S from TMEM (two lanes per head row, 48 key columns
 //     each), keep a running max (rescaling the output only when the max grows
 //     by more than 2^8) and write P (bf16) in the UMMA layout into the rope
 //     chunk of the tile's own stage (dead once S is done), so P is buffered
 //     with the stages at no extra shared memory;
-//   * O += P V on tcgen05 (M = 64, N = 2 x 256 latent columns, K = 64 keys),
+//   * O += P V on tcgen05 (M = 64, N = 2 x 256 latent columns, K = 96 keys),
 //     V read in place from the gathered tile as an MN-major operand.
 // The producers also pull the next tile's rows from HBM into L2
 // (prefetch.global.L2) while the current tile's copies land, and the MMA warp
@@ -37,7 +38,7 @@
 // log-sum-exp; mla_combine_kernel merges the shares.
 // TMEM (M = 64 operands occupy one 16-lane half of each 32-lane quarter):
 // lanes 0-15 hold Q (columns 0-287, two bf16 per column) and the two S buffers
-// (columns 288-415); lanes 16-31 hold O (columns 0-511).  Warp roles: warp 0
+// (from column 288); lanes 16-31 hold O (columns 0-511).  Warp roles: warp 0
 // MMA issuer / TMEM owner, warps 1-11 gather producers (all of them fill every
 // tile), warps 12-15 Q load, softmax and output.
 #include <cuda_bf16.h>
@@ -469,13 +470,26 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
         }
         vbits = ((lo >> c0) & 0xFFFFFFFFull) | (((hi >> (16 * half)) & 0xFFFFull) << 32);
       }
+      // Logits in the log2 domain, z = S * scale * log2(e) (packed multiplies);
+      // skipped or padding entries -inf, masked only in a tile that has any.
       float z[NC];
+      {
+        const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+#pragma unroll
+        for (int c = 0; c < NC; c += 2) {
+          const float2 zz = fmul2(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sc2);
+          z[c] = zz.x;
+          z[c + 1] = zz.y;
+        }
+      }
+      constexpr unsigned long long kAllCols = (1ull << NC) - 1ull;  // NC <= 48
+      if (!__all_sync(0xffffffffu, (vbits & kAllCols) == kAllCols)) {
+#pragma unroll
+        for (int c = 0; c < NC; ++c) z[c] = ((vbits >> c) & 1ull) ? z[c] : -INFINITY;
+      }
       float tmax = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < NC; ++c) {
-        z[c] = ((vbits >> c) & 1ull) ? __uint_as_float(sv[c]) * a.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, z[c]);
-      }
+      for (int c = 0; c < NC; c += 2) tmax = fmax3(tmax, z[c], z[c + 1]);
       tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));  // whole row (both halves)
       const float m_old = m_used;
       bool rescale = false;
@@ -483,19 +497,24 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
         rescale = (m_used != -INFINITY) && (j > 0);
         m_used = tmax;
       }
-      // P in bf16, rounded once; the normaliser sums the rounded values.
+      // P in bf16, rounded once; the normaliser sums the rounded values (two
+      // packed partial sums; the fp32 sum of the unrounded values feeds the
+      // LSE).  A row with no valid key yet has m = -inf and z = -inf: subtract
+      // 0 so that exp2 gives 0.
       uint32_t pk[NC / 2];
-      float tsum = 0.0f, tsum_exact = 0.0f;
+      const float m_sub = (m_used == -INFINITY) ? 0.0f : m_used;
+      const float2 m2 = make_float2(m_sub, m_sub);
+      float2 tsum2 = make_float2(0.0f, 0.0f), texact2 = make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int c = 0; c < NC; c += 2) {
-        const float p0 = (m_used == -INFINITY) ? 0.0f : fast_exp2(z[c] - m_used);
-        const float p1 = (m_used == -INFINITY) ? 0.0f : fast_exp2(z[c + 1] - m_used);
+        const float2 d = fsub2(make_float2(z[c], z[c + 1]), m2);
+        const float p0 = fast_exp2(d.x), p1 = fast_exp2(d.y);
         const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
-        const float2 br = __bfloat1622float2(b);
-        tsum += br.x + br.y;
-        tsum_exact += p0 + p1;
+        tsum2 = fadd2(tsum2, __bfloat1622float2(b));
+        texact2 = fadd2(texact2, make_float2(p0, p1));
         pk[c >> 1] = *reinterpret_cast<const uint32_t *>(&b);
       }
+      float tsum = tsum2.x + tsum2.y, tsum_exact = texact2.x + texact2.y;
       tsum += __shfl_xor_sync(0xffffffffu, tsum, 16);
       tsum_exact += __shfl_xor_sync(0xffffffffu, tsum_exact, 16);
       const float alpha = rescale ? fast_exp2(m_old - m_used) : 1.0f;
