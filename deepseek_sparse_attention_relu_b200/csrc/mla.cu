@@ -81,14 +81,20 @@ struct MlaCfg {
   static constexpr int PPW = (BK / 2 + N_PROD - 1) / N_PROD;  // 2-row groups per producer warp
   static constexpr int GPW = (BK / 4 + N_PROD - 1) / N_PROD;  // 4-row groups per producer warp
   static constexpr int OFF_KV = 0;
+  // Q is staged through shared memory once, from stage 1 on (idle until the
+  // second tile's gather): one 1,152-byte row every Q_PITCH bytes, so that the
+  // 16-byte reads of eight consecutive rows fall in distinct banks.
+  static constexpr int Q_PITCH = DIM * 2 + 16;
+  static constexpr int OFF_QSTAGE = OFF_KV + KV_BYTES;
   static constexpr int OFF_BAR = OFF_KV + STAGES * KV_BYTES;
-  static constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 1;
+  static constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 1 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_VALID = OFF_MISC + 64;      // [STAGES][N_PROD][2] key validity words (128 keys max)
   static constexpr int OFF_MEMB = OFF_VALID + STAGES * N_PROD * 16;  // [STAGES][64] per-query key masks (packed)
   static constexpr int SMEM_BYTES = OFF_MEMB + STAGES * 64 * 8 + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(S_COL + 2 * BK <= 512, "tensor memory budget");
+  static_assert(OFF_QSTAGE + HT * Q_PITCH <= OFF_BAR, "Q staging area");
   static_assert(BK % 32 == 0 && BK <= 128, "tile width");
 };
 
@@ -122,6 +128,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
   // barrier the parity of a phase two ahead would read as "not yet".
   uint64_t *p_full = s_full + 4;
   uint64_t *drain = p_full + STAGES;
+  uint64_t *q_copied = drain + 1;              // Q rows landed in the staging area (transaction bytes)
   unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + C::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
   unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + C::OFF_VALID);  // [STAGES][N_PROD][2]
@@ -169,6 +176,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
       mbar_init(&s_free[i], 4);
     }
     mbar_init(drain, 1);
+    mbar_init(q_copied, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -247,6 +255,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
       vlo |= __shfl_xor_sync(0xffffffffu, vlo, 16);
       vhi |= __shfl_xor_sync(0xffffffffu, vhi, 8);
       vhi |= __shfl_xor_sync(0xffffffffu, vhi, 16);
+      // Stage 1 on holds the staged Q rows until they are in tensor memory.
+      if (j == 1 && !mbar_wait(q_full, 0u, abort_flag)) { ok = false; break; }
       if (!mbar_wait(&kv_empty[st], ((j / STAGES) & 1) ^ 1u, abort_flag)) { ok = false; break; }
       // The stage's previous tile has been consumed (its softmax included).
       if (PACKED && pw == 0 && lane < nq) memb_s[st * 64 + lane] = cm;
@@ -397,13 +407,24 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
     const int row = quarter * 16 + r16;  // head within the CTA's group
     const unsigned lane_base = static_cast<unsigned>(quarter * 32) << 16;
     const int half = lane >> 4;          // which 32 of each 64 columns this thread's 16x32bx2 accesses cover
+    bool ok = true;
     {
-      // Q rows into tensor memory as the A operand of S = Q K^T: row `row`
-      // sits in lane quarter*32 + r16, dims 2c and 2c + 1 in column c.
-      // Thread halves take alternate 64-dim runs of the row (the 16x32bx2
+      // Q rows into tensor memory as the A operand of S = Q K^T, through the
+      // staging area: one bulk copy per valid row (two warps issue them), then
+      // row `row` goes to lane quarter*32 + r16, dims 2c and 2c + 1 in column
+      // c.  Thread halves take alternate 64-dim runs of the row (the 16x32bx2
       // store pairs them); rows past the tile's last valid row are zero.
-      const bool qv = row < row_limit;
-      const uint4 *src = reinterpret_cast<const uint4 *>(a.q) + (out_row0 + row) * (DIM / 8);
+      const unsigned qstage = smem_u32(smem + C::OFF_QSTAGE);
+      if (warp == WARP_SOFT0 && lane == 0) mbar_arrive_expect_tx(q_copied, static_cast<unsigned>(row_limit) * DIM * 2);
+      if (warp < WARP_SOFT0 + 2) {
+        const int qr = (warp - WARP_SOFT0) * 32 + lane;
+        if (qr < row_limit)
+          bulk_copy_g2s(qstage + qr * C::Q_PITCH, a.q + (out_row0 + qr) * DIM, DIM * 2, q_copied);
+      }
+      ok = mbar_wait(q_copied, 0u, abort_flag);
+      if (!ok) *abort_flag = 1;
+      const bool qv = ok && row < row_limit;
+      const uint8_t *src = smem + C::OFF_QSTAGE + row * C::Q_PITCH;
       const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
@@ -411,7 +432,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
         const int e0 = 128 * ch + 64 * half;  // first dim of this thread's run
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint4 v = qv ? src[e0 / 8 + k] : z4;
+          const uint4 v = qv ? *reinterpret_cast<const uint4 *>(src + (e0 + 8 * k) * 2) : z4;
           r[4 * k] = v.x;
           r[4 * k + 1] = v.y;
           r[4 * k + 2] = v.z;
@@ -424,7 +445,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
         const int e0 = 512 + 32 * half;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint4 v = qv ? src[e0 / 8 + k] : z4;
+          const uint4 v = qv ? *reinterpret_cast<const uint4 *>(src + (e0 + 8 * k) * 2) : z4;
           r[4 * k] = v.x;
           r[4 * k + 1] = v.y;
           r[4 * k + 2] = v.z;
@@ -438,12 +459,11 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
       if (lane == 0) mbar_arrive(q_full);
     }
     float m_used = -INFINITY, l = 0.0f, l_exact = 0.0f;  // l: sum of the bf16 P used; l_exact: fp32 sum for the LSE
-    bool ok = true;
     // This thread's NC of the tile's BK key columns: [32 half, 32 half + 32)
     // and, for 96-key tiles, also [64 + 16 half, 64 + 16 half + 16) (TMEM
     // half-split loads whose second half sits one load width further on).
     const int c0 = half * 32;
-    for (int j = 0; j < ntiles; ++j) {
+    for (int j = 0; ok && j < ntiles; ++j) {
       const int sb = j & 1;
       const int st = j % STAGES;
       if (!mbar_wait(&s_full[sb], (j >> 1) & 1u, abort_flag)) { ok = false; break; }
@@ -569,11 +589,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
       // split-key mode: this share's normalised fp32 output row
       const long long prow_idx = (static_cast<long long>(t - a.t0) * a.H + hg * HT + row) * a.nsplit + split;
       float *porow = split_mode ? a.part_o + prow_idx * LAT : nullptr;
-#pragma unroll 1
-      for (int ch = 0; ch < 8; ++ch) {
-        uint32_t ov[32];
-        tmem_ld_16x32bx2_x32(o_lat0 + lane_base + ch * 64, ov);
-        tmem_ld_wait();
+      // Normalise, convert and store 64 output columns of the row per step;
+      // the next step's tensor-memory load is in flight meanwhile.
+      auto emit = [&](int ch, const uint32_t (&ov)[32]) {
         const int d0 = 64 * ch + c0;  // this thread's 32 latent dims
         if (has_row && split_mode) {
           float4 *dst = reinterpret_cast<float4 *>(porow + d0);
@@ -593,6 +611,21 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
         }
+      };
+      uint32_t ova[32], ovb[32];
+      tmem_ld_16x32bx2_x32(o_lat0 + lane_base, ova);
+      tmem_ld_wait();
+      reg_fence(ova);
+#pragma unroll 1
+      for (int ch = 0; ch < 8; ch += 2) {
+        tmem_ld_16x32bx2_x32(o_lat0 + lane_base + (ch + 1) * 64, ovb);
+        emit(ch, ova);
+        tmem_ld_wait();
+        reg_fence(ovb);
+        if (ch + 2 < 8) tmem_ld_16x32bx2_x32(o_lat0 + lane_base + (ch + 2) * 64, ova);
+        emit(ch + 1, ovb);
+        tmem_ld_wait();
+        reg_fence(ova);
       }
       const float row_lse = l_exact > 0.0f ? (m_used + log2f(l_exact)) * 0.69314718055994530942f : -INFINITY;
       if (lane < 16 && has_row && split_mode) {
