@@ -87,7 +87,11 @@ struct MlaCfg {
   static constexpr int Q_PITCH = DIM * 2 + 16;
   static constexpr int OFF_QSTAGE = OFF_KV + KV_BYTES;
   static constexpr int OFF_BAR = OFF_KV + STAGES * KV_BYTES;
-  static constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 1 + 1;
+  // O += P V of a tile frees its stage in 32-key row groups (P of a group
+  // lies in the group's own rope rows), so the next gather into the stage
+  // starts while the later groups are still being multiplied.
+  static constexpr int NG = BK / 32;
+  static constexpr int NBAR = 1 + 4 * STAGES + 2 + 2 + 1 + 1 + NG * STAGES;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_VALID = OFF_MISC + 64;      // [STAGES][N_PROD][2] key validity words (128 keys max)
   static constexpr int OFF_MEMB = OFF_VALID + STAGES * N_PROD * 16;  // [STAGES][64] per-query key masks (packed)
@@ -129,6 +133,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
   uint64_t *p_full = s_full + 4;
   uint64_t *drain = p_full + STAGES;
   uint64_t *q_copied = drain + 1;              // Q rows landed in the staging area (transaction bytes)
+  uint64_t *grp_free = q_copied + 1;           // [STAGES][NG] O += P V done with the stage's 32-key row group
   unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + C::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
   unsigned long long *valid_s = reinterpret_cast<unsigned long long *>(smem + C::OFF_VALID);  // [STAGES][N_PROD][2]
@@ -177,6 +182,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
     }
     mbar_init(drain, 1);
     mbar_init(q_copied, 1);
+    for (int i = 0; i < STAGES * C::NG; ++i) mbar_init(&grp_free[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -257,34 +263,44 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
       vhi |= __shfl_xor_sync(0xffffffffu, vhi, 16);
       // Stage 1 on holds the staged Q rows until they are in tensor memory.
       if (j == 1 && !mbar_wait(q_full, 0u, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(&kv_empty[st], ((j / STAGES) & 1) ^ 1u, abort_flag)) { ok = false; break; }
-      // The stage's previous tile has been consumed (its softmax included).
-      if (PACKED && pw == 0 && lane < nq) memb_s[st * 64 + lane] = cm;
-      __syncwarp();
-      if (lane == 0) {
-        valid_s[(st * N_PROD + pw) * 2] = vlo;
-        valid_s[(st * N_PROD + pw) * 2 + 1] = vhi;
-        mbar_arrive(&valid_full[st]);
-      }
+      // Row group g (keys 32g .. 32g + 31) of the stage is refilled as soon as
+      // O += P V of the stage's previous tile is done with it.
       const unsigned stage_base = smem_u32(kv_s + st * KV_BYTES);
 #pragma unroll
-      for (int pr = 0; pr < 4; ++pr) {
-        const int c = 2 * pr + seg;
+      for (int g = 0; g < C::NG; ++g) {
+        if (!mbar_wait(&grp_free[st * C::NG + g], ((j / STAGES) & 1) ^ 1u, abort_flag)) { ok = false; break; }
+        if (g == 0) {
+          // The stage's previous tile has been consumed (its softmax included).
+          if (PACKED && pw == 0 && lane < nq) memb_s[st * 64 + lane] = cm;
+          __syncwarp();
+          if (lane == 0) {
+            valid_s[(st * N_PROD + pw) * 2] = vlo;
+            valid_s[(st * N_PROD + pw) * 2 + 1] = vhi;
+            mbar_arrive(&valid_full[st]);
+          }
+        }
 #pragma unroll
-        for (int i = 0; i < PPW; ++i) {
-          const int r = 2 * (pw + N_PROD * i) + sub2;
-          if (r < BK)
-            cp_async_16(stage_base + c * ATOM_BYTES + r * 128 + ((u ^ (r & 7)) << 4),
-                        kv + row_offset(kp[i]) + c * 128 + u * 16);
+        for (int pr = 0; pr < 4; ++pr) {
+          const int c = 2 * pr + seg;
+#pragma unroll
+          for (int i = 0; i < PPW; ++i) {
+            const int grp = pw + N_PROD * i;  // row pair
+            const int r = 2 * grp + sub2;
+            if (grp >= 16 * g && grp < 16 * g + 16 && r < BK)
+              cp_async_16(stage_base + c * ATOM_BYTES + r * 128 + ((u ^ (r & 7)) << 4),
+                          kv + row_offset(kp[i]) + c * 128 + u * 16);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < GPW; ++i) {
+          const int grp = pw + N_PROD * i;  // row quad
+          const int r = 4 * grp + sub4;
+          if (grp >= 8 * g && grp < 8 * g + 8 && r < BK)
+            cp_async_16(stage_base + 8 * ATOM_BYTES + r * 128 + ((u ^ (r & 7)) << 4),
+                        kv + row_offset(kq[i]) + 8 * 128 + u * 16);
         }
       }
-#pragma unroll
-      for (int i = 0; i < GPW; ++i) {
-        const int r = 4 * (pw + N_PROD * i) + sub4;
-        if (r < BK)
-          cp_async_16(stage_base + 8 * ATOM_BYTES + r * 128 + ((u ^ (r & 7)) << 4),
-                      kv + row_offset(kq[i]) + 8 * 128 + u * 16);
-      }
+      if (!ok) break;
       cp_async_arrive_noinc(&kv_full[st]);
       // Pull the next tile's rows from HBM into L2 now; its gather starts only
       // once its stage is consumed.
@@ -320,22 +336,24 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
     // below 2^18, so the 14-bit field never carries).
     const uint64_t k_desc0 = smem_desc_sw128(smem_u32(kv_s), 16, 1024);
     const uint64_t v_desc0 = smem_desc_sw128(smem_u32(kv_s), ATOM_BYTES, 1024);
-    // P (A of O += P V): 128-byte-swizzled rows for 64-key tiles; for 96-key
-    // tiles the no-swizzle core-matrix layout, which fits 64 x 96 bf16 in the
-    // 12 KB rope chunk (core matrices 128 B apart along K, 8-row groups
-    // BK / 8 * 128 B apart).
-    const uint64_t p_desc0 = BK == 64 ? smem_desc_sw128(smem_u32(kv_s + ROPE_OFF), 16, 1024)
-                                      : smem_desc_noswz(smem_u32(kv_s + ROPE_OFF), 128, BK / 8 * 128);
-    constexpr int P_KSTEP = BK == 64 ? 32 : 256;  // bytes between the P operands of consecutive 16-key steps
+    // P (A of O += P V) in the no-swizzle core-matrix layout, key-chunk major:
+    // the 8-row x 16-byte core matrix (row group rg, 8-key chunk kc) sits at
+    // kc * 1024 + rg * 128, so the P of keys 32g .. 32g + 31 fills exactly the
+    // rope rows of those keys (the rope chunk is dead once S = Q K^T is done).
+    const uint64_t p_desc0 = smem_desc_noswz(smem_u32(kv_s + ROPE_OFF), 1024, 128);
     auto issue_pv = [&](int jj) {
       const int s = jj % STAGES;
       const uint64_t so = static_cast<uint64_t>((s * KV_BYTES) >> 4);
 #pragma unroll
-      for (int ks = 0; ks < BK / 16; ++ks) {
-        const unsigned acc = (jj > 0 || ks > 0) ? 1u : 0u;
-        mma_bf16_ss(o_lat0, p_desc0 + so + ((ks * P_KSTEP) >> 4), v_desc0 + so + ((ks * 2048) >> 4), idesc_pv, acc);
-        mma_bf16_ss(o_lat1, p_desc0 + so + ((ks * P_KSTEP) >> 4),
-                    v_desc0 + so + ((4 * ATOM_BYTES + ks * 2048) >> 4), idesc_pv, acc);
+      for (int g = 0; g < C::NG; ++g) {
+#pragma unroll
+        for (int ks = 2 * g; ks < 2 * g + 2; ++ks) {
+          const unsigned acc = (jj > 0 || ks > 0) ? 1u : 0u;
+          mma_bf16_ss(o_lat0, p_desc0 + so + ((ks * 2048) >> 4), v_desc0 + so + ((ks * 2048) >> 4), idesc_pv, acc);
+          mma_bf16_ss(o_lat1, p_desc0 + so + ((ks * 2048) >> 4),
+                      v_desc0 + so + ((4 * ATOM_BYTES + ks * 2048) >> 4), idesc_pv, acc);
+        }
+        tc_commit(&grp_free[s * C::NG + g]);  // this group's V rows and P are read
       }
       tc_commit(&kv_empty[s]);
     };
@@ -566,10 +584,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
         for (int ch = 0; ch < NC / 8; ++ch) {
           const uint4 v = make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
           const int k = ch < 4 ? 4 * half + ch : 8 + 2 * half + (ch - 4);  // 8-key chunk of the tile
-          if constexpr (BK == 64)  // 128-byte-swizzled row
-            *reinterpret_cast<uint4 *>(pbase + row * 128 + ((k ^ (row & 7)) << 4)) = v;
-          else  // core matrix (row / 8, k), row row % 8 within it
-            *reinterpret_cast<uint4 *>(pbase + (row >> 3) * (BK / 8 * 128) + k * 128 + (row & 7) * 16) = v;
+          // core matrix (row / 8, k) at k * 1024 + (row / 8) * 128, row row % 8 within it
+          *reinterpret_cast<uint4 *>(pbase + k * 1024 + row * 16) = v;
         }
       }
       fence_proxy_async_smem();
