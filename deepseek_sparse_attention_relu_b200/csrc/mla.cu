@@ -607,6 +607,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
       float *porow = split_mode ? a.part_o + prow_idx * LAT : nullptr;
       // Normalise, convert and store 64 output columns of the row per step;
       // the next step's tensor-memory load is in flight meanwhile.
+      // Rows are 1,024 bytes and each thread's 32 dims start 64-byte aligned:
+      // 32-byte stores work whenever the output itself is 32-byte aligned.
+      const bool out32 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
       auto emit = [&](int ch, const uint32_t (&ov)[32]) {
         const int d0 = 64 * ch + c0;  // this thread's 32 latent dims
         if (has_row && split_mode) {
@@ -623,9 +626,14 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(MlaArgs a) {
                 __floats2bfloat162_rn(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
             pkd[e] = *reinterpret_cast<const uint32_t *>(&b);
           }
-          uint4 *dst = reinterpret_cast<uint4 *>(orow + d0);
+          if (out32) {  // two 32-byte stores: whole 32-byte sectors, half the store requests
+            st_global_v8(orow + d0, pkd);
+            st_global_v8(orow + d0 + 16, pkd + 8);
+          } else {
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + d0);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+          }
         }
       };
       uint32_t ova[32], ovb[32];
