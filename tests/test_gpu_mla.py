@@ -99,6 +99,26 @@ def test_single_key_is_exact_and_no_key_is_zero():
     assert np.all(out[2] == 0.0) and np.all(np.isneginf(lse[2]))
 
 
+def test_output_alignment_16_and_32_bytes():
+    """Output rows go out as 32-byte stores when the output is 32-byte aligned and as 16-byte stores when it is
+    only 16-byte aligned: the bits must not depend on which."""
+    N, L, H, topk = 3000, 5, 64, 256
+    q, kv = make(N, L, H, seed=13)
+    idx = torch.from_numpy(random_selection(N, L, topk, seed=13)).cuda()
+    q, kv = q.cuda(), kv.cuda()
+    ws = dsa.alloc_workspace(dsa.dsa_sparse_mla_workspace(L, H, topk), torch.device("cuda"))
+    ref = torch.empty((L, H, 512), dtype=torch.bfloat16, device="cuda")
+    assert ref.data_ptr() % 32 == 0
+    dsa.dsa_sparse_mla_prefill(q, kv, idx, 1 / math.sqrt(192), ref, workspace=ws)
+    buf = torch.full((L * H * 512 + 8,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    shifted = buf[8:].view(L, H, 512)  # 16 bytes past a 32-byte boundary
+    assert shifted.data_ptr() % 32 == 16
+    dsa.dsa_sparse_mla_prefill(q, kv, idx, 1 / math.sqrt(192), shifted, workspace=ws)
+    assert dsa.dsa_workspace_status(ws) == 0
+    assert torch.equal(ref, shifted)
+    assert torch.isnan(buf[:8]).all()  # nothing written before the output
+
+
 def test_full_selection_matches_dense_causal():
     """top-k covering every visible key: the sparse path equals dense causal attention (mlx-lm PR #1997 tests)."""
     N = L = 300
