@@ -77,6 +77,17 @@ def test_ragged_topk_and_padding():
     check(q, kv, idx, 1 / math.sqrt(192))
 
 
+@pytest.mark.parametrize("topk,pad", [(32, 0), (33, 0), (95, 0), (96, 0), (97, 0), (160, 31), (192, 0), (193, 64),
+                                      (288, 1), (2047, 0)])
+def test_tile_and_group_boundaries(topk, pad):
+    """Selections ending at, just before and just after a 32-key release group and a 96-key tile, with and
+    without -1 padding: every key lands in the right row group of the right stage."""
+    N, L, H = 4096, 4, 64
+    q, kv = make(N, L, H, seed=topk)
+    idx = random_selection(N, L, topk, seed=topk + 1, pad=pad)
+    check(q, kv, idx, 1 / math.sqrt(192))
+
+
 def test_unsorted_indices_and_large_scale():
     N, L, topk = 4096, 6, 512
     q, kv = make(N, L, 64, seed=5, lat_std=1.0, rope_std=1.0)
