@@ -12,8 +12,9 @@
 // Index -1 marks a skipped entry (llama.cpp PR #25917, discussion).
 //
 // B200 mapping.  One CTA per (query, group of 64 heads).  Q lives in tensor
-// memory for the whole CTA: the softmax warps copy its 64 x 576 bf16 rows
-// there once, and S = Q K^T reads its A operand from tensor memory, so shared
+// memory for the whole CTA: its 64 x 576 bf16 rows arrive by bulk copies in
+// the still idle second stage and the softmax warps move them into tensor
+// memory once, and S = Q K^T reads its A operand from there, so shared
 // memory holds only gathered keys (two 108 KB stages of 96-key tiles; the
 // packed variant uses three 72 KB stages of 64 keys) and the S MMAs read only
 // the key tile from it.  Per tile:
@@ -29,7 +30,9 @@
 //     chunk of the tile's own stage (dead once S is done), so P is buffered
 //     with the stages at no extra shared memory;
 //   * O += P V on tcgen05 (M = 64, N = 2 x 256 latent columns, K = 96 keys),
-//     V read in place from the gathered tile as an MN-major operand.
+//     V read in place from the gathered tile as an MN-major operand; it
+//     commits per 32-key group, and the producers refill each group of the
+//     stage as soon as its MMAs are done.
 // The producers also pull the next tile's rows from HBM into L2
 // (prefetch.global.L2) while the current tile's copies land, and the MMA warp
 // polls its barriers with the non-suspending mbarrier.test_wait.  Split-key
