@@ -85,8 +85,10 @@ const char *dsa_last_error_string(void);
  * Workspace (bytes) that dsa_indexer_topk needs for these sizes.  A larger
  * buffer is fine.  A smaller one that still holds the fixed part shrinks the
  * per-query candidate capacity; queries whose candidates do not fit are then
- * resolved by the exact fallback (slower, same result).  Returns 0 for
- * invalid sizes.
+ * resolved by the exact fallback (slower, same result).  The fixed part holds
+ * one N-score row per CTA of the exact fallback, one CTA per SM of the
+ * current device (at least 16, at most one per query of a block), so the size
+ * depends on the device queried.  Returns 0 for invalid sizes.
  */
 size_t dsa_indexer_topk_workspace(int L, int N, int H_I, int D_I, int topk, dsa_dtype_t dtype);
 
