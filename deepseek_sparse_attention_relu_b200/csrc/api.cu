@@ -18,7 +18,7 @@ using namespace dsa;
 
 constexpr int kDefaultQueryBlock = 1024;  // mlx-lm PR #1997: query blocks of 1,024
 constexpr int kSamples = 4096;            // strided key sample per query block
-constexpr int kFallbackSlots = 16;        // CTAs (and score rows) of the exact fallback, at least
+constexpr int kFallbackSlots = 16;        // CTAs of the exact fallback: at least this many (exactly, without a workspace)
 constexpr int kMinCap = 8192;             // default candidate capacity per query
 constexpr int kMaxTopk = 4096;
 constexpr size_t kHeaderBytes = 256;      // status word, fallback counters, selection totals
@@ -94,17 +94,17 @@ int query_block_size(int L, int query_block, int H_I) {
   return static_cast<int>(std::min<long long>(L, qb));
 }
 
-// CTAs (and dense score rows) of the exact fallback for a block of QB
-// queries: one per SM, so that many fallback queries are rescored at once
-// (each CTA takes one query at a time), and never more than the block has.
-int fallback_slots(int QB) {
-  return std::max(1, std::min(QB, std::max(kFallbackSlots, sm_count())));
-}
+// CTAs of the exact fallback: one per SM (at least kFallbackSlots), so that
+// many fallback queries are rescored at once and a few are split over all
+// of them.  Its dense score rows: one per CTA, but never more than a block
+// has queries (a query's chunks share its row).
+int fallback_ctas() { return std::max(kFallbackSlots, sm_count()); }
+size_t fallback_rows(int QB, int fb_ctas) { return static_cast<size_t>(std::max(1, std::min(QB, fb_ctas))); }
 
 // Fixed part of the indexer workspace (everything but the candidate lists).
-size_t idx_fixed_bytes(int QB, int N, int fb_slots) {
-  return kHeaderBytes + 5 * align256(static_cast<size_t>(QB) * 4) + 2 * align256((QB + 2) * sizeof(int)) +
-         align256(static_cast<size_t>(QB) * kSamples * 4) + align256(static_cast<size_t>(fb_slots) * N * 4);
+size_t idx_fixed_bytes(int QB, int N, int fb_ctas) {
+  return kHeaderBytes + 6 * align256(static_cast<size_t>(QB) * 4) + 2 * align256((QB + 2) * sizeof(int)) +
+         align256(static_cast<size_t>(QB) * kSamples * 4) + align256(fallback_rows(QB, fb_ctas) * N * 4);
 }
 
 struct IdxWorkspace {
@@ -114,18 +114,19 @@ struct IdxWorkspace {
   unsigned *tau;
   int *cand_count;
   int *fb_list;
+  int *fb_done;
   float *dense;
   float *fb_scratch;
   unsigned long long *cand;
   int *rlo, *rhi;                 // [QB] clamped per-query key ranges (ranges mode)
   int *grp_tile0, *grp_start;     // per-group tile windows (ranges mode)
   int cap;
-  int fb_slots;                   // rows of fb_scratch = CTAs of the exact fallback
+  int fb_ctas;                    // CTAs of the exact fallback (fb_scratch holds fallback_rows rows)
 };
 
-bool carve_idx_ws(void *ws, size_t bytes, int QB, int N, int fb_slots, IdxWorkspace *o) {
-  const size_t fixed = idx_fixed_bytes(QB, N, fb_slots);
-  o->fb_slots = fb_slots;
+bool carve_idx_ws(void *ws, size_t bytes, int QB, int N, int fb_ctas, IdxWorkspace *o) {
+  const size_t fixed = idx_fixed_bytes(QB, N, fb_ctas);
+  o->fb_ctas = fb_ctas;
   if (ws == nullptr || bytes < fixed + static_cast<size_t>(QB) * 8) return false;
   uint8_t *p = static_cast<uint8_t *>(ws);
   o->status = reinterpret_cast<unsigned *>(p);
@@ -138,6 +139,8 @@ bool carve_idx_ws(void *ws, size_t bytes, int QB, int N, int fb_slots, IdxWorksp
   p += align256(static_cast<size_t>(QB) * 4);
   o->fb_list = reinterpret_cast<int *>(p);
   p += align256(static_cast<size_t>(QB) * 4);
+  o->fb_done = reinterpret_cast<int *>(p);
+  p += align256(static_cast<size_t>(QB) * 4);
   o->rlo = reinterpret_cast<int *>(p);
   p += align256(static_cast<size_t>(QB) * 4);
   o->rhi = reinterpret_cast<int *>(p);
@@ -149,7 +152,7 @@ bool carve_idx_ws(void *ws, size_t bytes, int QB, int N, int fb_slots, IdxWorksp
   o->dense = reinterpret_cast<float *>(p);
   p += align256(static_cast<size_t>(QB) * kSamples * 4);
   o->fb_scratch = reinterpret_cast<float *>(p);
-  p += align256(static_cast<size_t>(fb_slots) * N * 4);
+  p += align256(fallback_rows(QB, fb_ctas) * N * 4);
   o->cand = reinterpret_cast<unsigned long long *>(p);
   const size_t room = (bytes - fixed) / (static_cast<size_t>(QB) * 8);
   o->cap = static_cast<int>(std::min<size_t>(room, 1u << 30));
@@ -270,6 +273,7 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
   sa.cand_count = ws.cand_count;
   sa.fb_list = ws.fb_list;
   sa.fb_counters = ws.fb_counters;
+  sa.fb_done = ws.fb_done;
   sa.status = ws.status;
   sa.stats = ws.stats;
   sa.topk_idx = p.topk_idx;
@@ -319,10 +323,11 @@ dsa_status_t run_indexer_block(const IndexerProblem &p, const CUtensorMap &tq, c
   fa.dense_ld = p.N;
   fa.fb_list = ws.fb_list;
   fa.fb_counters = ws.fb_counters;
+  fa.fb_done = ws.fb_done;
   fa.topk_idx = p.topk_idx + static_cast<long long>(t0) * p.topk;
   fa.topk_score = p.topk_score ? p.topk_score + static_cast<long long>(t0) * p.topk : nullptr;
   fa.topk = p.topk;
-  if (!cuda_ok(launch_indexer(tq, tk, fa, p.D_I, p.H_I, p.fp8, kIdxFallback, ws.fb_slots, stream)))
+  if (!cuda_ok(launch_indexer(tq, tk, fa, p.D_I, p.H_I, p.fp8, kIdxFallback, ws.fb_ctas, stream)))
     return DSA_ERR_CUDA;
   if (!mark(ev, 5, stream)) return DSA_ERR_CUDA;
   return DSA_OK;
@@ -522,7 +527,7 @@ size_t dsa_indexer_topk_workspace(int L, int N, int H_I, int D_I, int topk, dsa_
   if (L <= 0 || N <= 0 || H_I <= 0 || D_I <= 0 || topk <= 0) return 0;
   (void)dtype;
   const int QB = query_block_size(L, 0, H_I);
-  return idx_fixed_bytes(QB, N, fallback_slots(QB)) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
+  return idx_fixed_bytes(QB, N, fallback_ctas()) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
 }
 
 }  // extern "C"
@@ -542,7 +547,7 @@ dsa_status_t indexer_topk_impl(const void *q_idx, const void *k_idx, int64_t ldk
   if (st != DSA_OK) return st;
   const int QB = query_block_size(L, 0, H_I);
   IdxWorkspace ws;
-  if (!carve_idx_ws(workspace, workspace_bytes, QB, N, fallback_slots(QB), &ws)) return DSA_ERR_WORKSPACE;
+  if (!carve_idx_ws(workspace, workspace_bytes, QB, N, fallback_ctas(), &ws)) return DSA_ERR_WORKSPACE;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   CUtensorMap tq, tk;
   if (!make_indexer_maps(p, &tq, &tk)) return DSA_ERR_CUDA;
@@ -601,7 +606,7 @@ size_t dsa_prefill_chunk_workspace(int L, int N, int H_I, int D_I, int H, int to
   if (L <= 0 || N <= 0 || H_I <= 0 || D_I <= 0 || H <= 0 || topk <= 0) return 0;
   (void)dtype;
   const int QB = query_block_size(L, query_block, H_I);
-  size_t bytes = idx_fixed_bytes(QB, N, fallback_slots(QB)) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
+  size_t bytes = idx_fixed_bytes(QB, N, fallback_ctas()) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
   if (!want_topk_out) bytes += align256(static_cast<size_t>(QB) * topk * 4);
   const size_t extra = attention_scratch_bytes(L, QB, H, topk);
   if (extra > 0) bytes += extra + 256;
@@ -634,7 +639,7 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, int64_t ld
   UnionWorkspace uw;
   const size_t ub = attention_scratch_bytes(L, QB, H, topk);
   const size_t idx_need =
-      idx_fixed_bytes(QB, N, fallback_slots(QB)) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
+      idx_fixed_bytes(QB, N, fallback_ctas()) + align256(static_cast<size_t>(QB) * default_cap(topk) * 8);
   if (ub > 0 && workspace != nullptr && idx_bytes >= ub + idx_need) {
     const size_t off = (idx_bytes - ub) & ~static_cast<size_t>(255);
     uw.base = static_cast<uint8_t *>(workspace) + off;
@@ -653,7 +658,7 @@ dsa_status_t prefill_chunk_impl(const void *q_idx, const void *k_idx, int64_t ld
   st = check_mla_args(mp);
   if (st != DSA_OK) return st;
   IdxWorkspace ws;
-  if (!carve_idx_ws(workspace, idx_bytes, QB, N, fallback_slots(QB), &ws)) return DSA_ERR_WORKSPACE;
+  if (!carve_idx_ws(workspace, idx_bytes, QB, N, fallback_ctas(), &ws)) return DSA_ERR_WORKSPACE;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   CUtensorMap tq, tk;
   if (!make_indexer_maps(ip, &tq, &tk)) return DSA_ERR_CUDA;

@@ -48,11 +48,16 @@ struct IndexerArgs {
   int total_tiles;                // sum over query groups of their 128-key tiles
   int pilot;                      // 1 = PILOT mode
   // FALLBACK mode: the CTAs take the queries of fb_list[0 .. fb_counters[0])
-  // one at a time (fb_counters[1] hands them out), score every visible key of
-  // the query into their own dense row of `dense` (dense_ld = N floats per
-  // CTA) and select its exact top-k into topk_idx / topk_score.
+  // (fb_counters[1] hands out jobs), score every visible key of the query into
+  // a dense row of `dense` (dense_ld = N floats per row) and select its exact
+  // top-k into topk_idx / topk_score.  With at least as many CTAs as queries,
+  // a query's key tiles are split into gridDim.x / count chunks, one job each,
+  // into row = the query's position in fb_list, and the CTA that completes its
+  // last chunk (fb_done counts them) selects; otherwise a job is a whole query
+  // and a CTA uses its own row blockIdx.x.
   const int *fb_list;             // [Lb] queries of the block, as positions tl
   int *fb_counters;               // [0] = count, [1] = next
+  int *fb_done;                   // [Lb] chunks done per fallback query (zeroed by the selection)
   int32_t *topk_idx;              // [Lb, topk] rows of the block's queries
   float *topk_score;              // [Lb, topk] or nullptr
   int topk;
@@ -106,6 +111,7 @@ struct SelectArgs {
   int *cand_count;                // [Lb]
   int *fb_list;                   // [Lb] queries that need the exact fallback
   int *fb_counters;               // [0] = count, [1] = next
+  int *fb_done;                   // [Lb] chunk counters of the fallback queries (zeroed here)
   unsigned *status;
   SelectionStats *stats;          // totals over the call (workspace header)
   int32_t *topk_idx;              // [L, topk] whole chunk

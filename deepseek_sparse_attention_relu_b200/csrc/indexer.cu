@@ -223,6 +223,8 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
   unsigned *tmem_slot = reinterpret_cast<unsigned *>(smem + C::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
   volatile int *job_s = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 12);  // FALLBACK: current query
+  // FALLBACK: [0] score row, [1] chunk, [2] chunks per query, [3] position in fb_list, [4] select flag
+  volatile int *job_meta = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 16);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -311,20 +313,42 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     // ---- the tiles of this round: the CTA's share of the block (one round),
     // or one fallback query at a time.
     TileCursor c;
-    int job_tl = -1, job_lo = 0, job_hi = 0;
+    int job_tl = -1, job_lo = 0, job_hi = 0, job_row = 0, job_cpq = 1, job_pos = 0;
     if constexpr (FB) {
       if (threadIdx.x == 0) {
         int j = -1;
         if (!*abort_flag) {
+          // Fewer queries than CTAs: each query's tiles are split into
+          // gridDim.x / count chunks (one job each) so that all CTAs work.
+          const int nfb = *reinterpret_cast<volatile int *>(&a.fb_counters[0]);  // >= 1 here
+          const int cpq = nfb < static_cast<int>(gridDim.x) ? static_cast<int>(gridDim.x) / nfb : 1;
           const int n = atomicAdd(&a.fb_counters[1], 1);
-          if (n < *reinterpret_cast<volatile int *>(&a.fb_counters[0])) j = a.fb_list[n];
+          if (n < nfb * cpq) {
+            const int pos = n / cpq;
+            j = a.fb_list[pos];
+            job_meta[0] = cpq > 1 ? pos : static_cast<int>(blockIdx.x);
+            job_meta[1] = n - pos * cpq;
+            job_meta[2] = cpq;
+            job_meta[3] = pos;
+          }
         }
         *job_s = j;
       }
       __syncthreads();
       job_tl = *job_s;
       if (job_tl < 0) break;
+      job_row = job_meta[0];
+      job_cpq = job_meta[2];
+      job_pos = job_meta[3];
       c = idx_cursor_job<RANGES>(a, job_tl, C::QG, job_lo, job_hi);
+      if (job_cpq > 1) {  // this job's share of the query's tiles
+        const int per = (c.ntiles_g + job_cpq - 1) / job_cpq;
+        const int first = min(c.ntiles_g, job_meta[1] * per);
+        const int len = min(per, c.ntiles_g - first);
+        c.tile0 += first;
+        c.ntiles_g = len;
+        c.left = len;
+      }
       e_prev_g = -1;  // every job loads its group's weights afresh
     } else {
       if (round > 0) break;
@@ -463,7 +487,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
             if (tl < a.Lb && key < a.n_keys) a.dense[static_cast<long long>(tl) * a.dense_ld + key] = score;
           } else if (FB) {
             if (tl == job_tl && key >= job_lo && key < job_hi)
-              a.dense[static_cast<long long>(blockIdx.x) * a.dense_ld + (key - job_lo)] = score;
+              a.dense[static_cast<long long>(job_row) * a.dense_ld + (key - job_lo)] = score;
           } else {
             const bool vis = RANGES ? (key >= lo_w[qq] && key < hi_w[qq]) : (key <= a.q_pos0 + tl);
             const bool pass = (tl < a.Lb) && vis && (score >= tau_w[qq]);
@@ -572,13 +596,26 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
     }
 
     if constexpr (FB) {
-      // The job's dense row is complete (every epilogue write precedes the
-      // barrier); the whole CTA selects its exact top-k from it.
+      // The job's scores are written (every epilogue write precedes the
+      // fence and the barrier).  A whole query: the CTA selects its exact
+      // top-k from the row.  A chunk: the CTA that completes the query's last
+      // chunk does, once every chunk's scores are visible.
+      __threadfence();
       __syncthreads();
-      if (!*abort_flag) {
+      bool select_now = true;
+      if (job_cpq > 1) {
+        if (threadIdx.x == 0) {
+          const int done = atomicAdd(&a.fb_done[job_pos], 1);
+          __threadfence();
+          job_meta[4] = done == job_cpq - 1 ? 1 : 0;
+        }
+        __syncthreads();
+        select_now = job_meta[4] != 0;
+      }
+      if (select_now && !*abort_flag) {
         const int need = min(a.topk, job_hi - job_lo);
         DenseSelectSmem *sm = reinterpret_cast<DenseSelectSmem *>(smem + C::OFF_STG);
-        select_dense_row(a.dense + static_cast<long long>(blockIdx.x) * a.dense_ld, job_lo, job_hi - job_lo, need,
+        select_dense_row(a.dense + static_cast<long long>(job_row) * a.dense_ld, job_lo, job_hi - job_lo, need,
                          a.topk, a.topk_idx + static_cast<long long>(job_tl) * a.topk,
                          a.topk_score ? a.topk_score + static_cast<long long>(job_tl) * a.topk : nullptr, a.status,
                          sm);

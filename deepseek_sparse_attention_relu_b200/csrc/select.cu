@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     if (threadIdx.x == 0) {
       const int pos = atomicAdd(&a.fb_counters[0], 1);
       a.fb_list[pos] = tl;
+      a.fb_done[pos] = 0;
     }
     return;
   }

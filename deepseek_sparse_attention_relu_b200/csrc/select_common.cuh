@@ -12,7 +12,9 @@ namespace dsa {
 // Block-wide MSB-first radix select.  Among n unique keys (fetch(i), i < n) find
 // (prefix, mask) such that exactly `need` keys satisfy (key & mask) >= prefix,
 // i.e. key >= prefix.  1 <= need <= n.  Every thread of the block must call it.
-template <typename KeyT, typename Fetch>
+// UNROLL > 1 keeps that many keys per thread in flight in the histogram passes
+// (for keys read from global memory).
+template <typename KeyT, int UNROLL = 1, typename Fetch>
 __device__ void block_radix_select(Fetch fetch, int n, int need, KeyT &prefix_out, KeyT &mask_out,
                                    unsigned *hist, unsigned *misc) {
   constexpr int BITS = sizeof(KeyT) * 8;
@@ -21,7 +23,19 @@ __device__ void block_radix_select(Fetch fetch, int n, int need, KeyT &prefix_ou
   for (int shift = BITS - 8; shift >= 0; shift -= 8) {
     for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[b] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int bd = static_cast<int>(blockDim.x);
+    int i = threadIdx.x;
+    if constexpr (UNROLL > 1) {
+      for (; i + (UNROLL - 1) * bd < n; i += UNROLL * bd) {
+        KeyT kk[UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) kk[u] = fetch(i + u * bd);
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u)
+          if ((kk[u] & mask) == prefix) atomicAdd(&hist[static_cast<unsigned>(kk[u] >> shift) & 255u], 1u);
+      }
+    }
+    for (; i < n; i += bd) {
       const KeyT k = fetch(i);
       if ((k & mask) == prefix) atomicAdd(&hist[static_cast<unsigned>(k >> shift) & 255u], 1u);
     }
@@ -107,24 +121,25 @@ struct DenseSelectSmem {
 // DEV_OVERFLOW.
 __device__ __forceinline__ void select_dense_row(const float *scores, int lo, int nvis, int need, int topk,
                                                  int32_t *out, float *osc, unsigned *status, DenseSelectSmem *sm) {
-  auto key_of = [&](int j) {
-    return (static_cast<unsigned long long>(float_order_key(scores[j])) << 32) |
+  auto key_of = [&](int j) {  // L2 reads: other CTAs may have written parts of the row
+    return (static_cast<unsigned long long>(float_order_key(__ldcg(scores + j))) << 32) |
            static_cast<unsigned>(~static_cast<unsigned>(lo + j));
   };
   unsigned long long prefix = 0, mask = 0;
-  if (nvis > need) block_radix_select<unsigned long long>(key_of, nvis, need, prefix, mask, sm->hist, sm->misc);
+  if (nvis > need) block_radix_select<unsigned long long, 4>(key_of, nvis, need, prefix, mask, sm->hist, sm->misc);
   // Ordered compaction: each thread takes a contiguous run of keys, so the
   // block prefix sum of the per-thread counts gives every winner its slot.
   const int per = (nvis + blockDim.x - 1) / blockDim.x;
   const int j0 = threadIdx.x * per, j1 = min(nvis, j0 + per);
   int mine = 0;
+#pragma unroll 4
   for (int j = j0; j < j1; ++j) mine += key_of(j) >= prefix ? 1 : 0;
   int pos = block_exclusive_scan(mine, sm->warp_tot, &sm->total);
   for (int j = j0; j < j1; ++j) {
     if (key_of(j) >= prefix) {
       if (pos < need) {
         out[pos] = lo + j;
-        if (osc) osc[pos] = scores[j];
+        if (osc) osc[pos] = __ldcg(scores + j);
       }
       ++pos;
     }

@@ -154,10 +154,11 @@ dsa_status_t dsa_indexer_topk_ranges(const void *q_idx, const void *k_idx, int64
  *
  *   - Limit: problems whose scratch exceeds 16 MiB at 64-query blocks are
  *     rejected with DSA_ERR_WORKSPACE before anything is launched (with
- *     top-k <= 2048 that admits N up to about 180,000 cached keys).
+ *     top-k <= 2048 that admits N up to about 180,000 cached keys; calls of
+ *     fewer than 16 queries hold fewer fallback score rows and admit more).
  *   - The first call on each device (each CUDA context: again after a device
- *     reset) looks up the array's device address with cudaGetSymbolAddress;
- *     make that first call before any stream capture.
+ *     reset) looks up the array's device address with cudaGetSymbolAddress,
+ *     a synchronous runtime query.
  *   - No cudaMalloc or cudaFree, and no allocating library call, is made.
  *   - Every call on a device shares the one array, which keeps the previous
  *     call's contents; the call clears what must start at zero.  Calls that

@@ -49,8 +49,9 @@ def test_noalloc_matches_workspace_entry_point(cfg):
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
+    # 64 queries: a full 64-query block, whose 16 fallback score rows of N floats alone fill the fixed scratch
     dev = torch.device("cuda")
-    N, L = 262144, 8
+    N, L = 262144, 64
     q = torch.zeros(L, 32, 128, dtype=torch.bfloat16, device=dev)
     k = torch.zeros(N, 128, dtype=torch.bfloat16, device=dev)
     w = torch.zeros(L, 32, dtype=torch.float32, device=dev)
