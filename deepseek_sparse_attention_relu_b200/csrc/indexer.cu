@@ -618,7 +618,7 @@ __global__ void __launch_bounds__(IdxCfg<DI, HI, FP8>::THREADS, 1)
         select_dense_row(a.dense + static_cast<long long>(job_row) * a.dense_ld, job_lo, job_hi - job_lo, need,
                          a.topk, a.topk_idx + static_cast<long long>(job_tl) * a.topk,
                          a.topk_score ? a.topk_score + static_cast<long long>(job_tl) * a.topk : nullptr, a.status,
-                         sm);
+                         sm, reinterpret_cast<unsigned *>(smem + C::OFF_Q), C::OFF_STG / 4);  // query + key stages are idle
       }
     }
   }
