@@ -43,6 +43,10 @@ def test_workspace_sizes(lib):
     b = lib.dsa_indexer_topk_workspace(4096, 131072, 32, 128, 2048, 0)
     assert a > 1024 * 8192 * 8 and a == b  # query blocks of 1,024 bound the workspace
     assert lib.dsa_indexer_topk_workspace(0, 10, 32, 128, 8, 0) == 0
+    # one query (decode): one exact-fallback score row and one candidate list, however many fallback CTAs run
+    assert lib.dsa_indexer_topk_workspace(1, 131072, 32, 128, 2048, 0) < (1 << 20)
+    # a 1,024-query block holds at least 16 fallback score rows of N floats
+    assert a > 16 * 131072 * 4 + 1024 * 8192 * 8
     c = lib.dsa_prefill_chunk_workspace(1024, 131072, 32, 128, 64, 2048, 0, 0, 0)
     d = lib.dsa_prefill_chunk_workspace(1024, 131072, 32, 128, 64, 2048, 0, 0, 1)
     assert c - d >= 1024 * 2048 * 4
